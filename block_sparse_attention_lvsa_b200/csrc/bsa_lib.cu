@@ -1,0 +1,289 @@
+// bsa_lib.cu - C ABI of libbsa.so (declared in include/bsa.h).
+//
+// Host side of every call: argument validation (before anything is
+// enqueued), TMA tensor-map encoding, workspace carving and kernel launches
+// on the caller's stream.  The library allocates no memory and never
+// synchronises except in bsa_get_device_status.  Everything is one
+// translation unit so the per-device status word is a single symbol.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "ptx.cuh"
+#include "lvsa_index.cuh"
+#include "losa_select.cuh"
+#include "attn_fwd.cuh"
+
+namespace {
+
+using namespace bsa;
+
+constexpr long long kWaitLimitNs = 1500000000LL;   // 1.5 s per device-side wait
+constexpr int kMaxDevices = 64;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D view (d, H, N) of a bf16 [N, H, d] tensor; box (64, 1, 128), 128B swizzle.
+bool make_qkv_map(CUtensorMap* m, const void* ptr, int N, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int n_tiles(int N) { return (N + 127) / 128; }
+
+int check_qkv(const void* q, const void* k, const void* v, int N, int H, int d, const void* o, const float* lse) {
+  if (!q || !k || !v || !o || !lse) return BSA_ERR_ARG;
+  if (N < 1 || H < 1 || H > 65535) return BSA_ERR_ARG;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * H * d >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return BSA_ERR_ARG;
+  return BSA_OK;
+}
+
+template <int D, bool MASS>
+int launch_attn(const void* q, const void* k, const void* v, int N, int H, const AttnParams& prm,
+                cudaStream_t st) {
+  using L = AttnSmem<D, MASS>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(attn_tile_kernel<D, MASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L::kAlloc)) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!make_qkv_map(&mq, q, N, H, D) || !make_qkv_map(&mk, k, N, H, D) || !make_qkv_map(&mv, v, N, H, D))
+    return BSA_ERR_CUDA;
+  dim3 grid(prm.nB, H);
+  attn_tile_kernel<D, MASS><<<grid, kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
+int launch_attn_any(int d, bool mass, const void* q, const void* k, const void* v, int N, int H,
+                    const AttnParams& prm, cudaStream_t st) {
+  if (d == 128) return mass ? launch_attn<128, true>(q, k, v, N, H, prm, st)
+                            : launch_attn<128, false>(q, k, v, N, H, prm, st);
+  return mass ? launch_attn<64, true>(q, k, v, N, H, prm, st) : launch_attn<64, false>(q, k, v, N, H, prm, st);
+}
+
+AttnParams base_params(int N, int H, float scale, void* o, float* lse) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.N = N;
+  p.H = H;
+  p.nB = n_tiles(N);
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.wait_limit_ns = kWaitLimitNs;
+  return p;
+}
+
+// Workspace layout for LVSA frame indexes.
+struct LvsaWs {
+  size_t fbits, cnt, idx, flag, total;
+};
+LvsaWs lvsa_ws_layout(int N, int T) {
+  const size_t nB = static_cast<size_t>(n_tiles(N));
+  const size_t TW = static_cast<size_t>((T + 31) / 32);
+  LvsaWs w;
+  w.fbits = 0;
+  w.cnt = round_up(w.fbits + static_cast<size_t>(T) * TW * 4, 256);
+  w.idx = round_up(w.cnt + nB * 4, 256);
+  w.flag = round_up(w.idx + nB * nB * 4, 256);
+  w.total = round_up(w.flag + nB * nB, 256);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bsa_version(void) { return "bsa-b200 0.1 (sm_100a)"; }
+
+const char* bsa_status_string(int s) {
+  switch (s) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_WARN_OVER_BUDGET: return "BSA_WARN_OVER_BUDGET";
+    case BSA_ERR_ARG: return "BSA_ERR_ARG";
+    case BSA_ERR_SHAPE: return "BSA_ERR_SHAPE";
+    case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+    case BSA_ERR_INDEX_RANGE: return "BSA_ERR_INDEX_RANGE";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
+    default: return "BSA_UNKNOWN_STATUS";
+  }
+}
+
+int lvsa_build_index(int T, int T_per, int W, int C, int step, int32_t* frames, int32_t* counts, void* stream) {
+  if (T < 1 || T > kMaxFrames || T_per < 1 || W < 1 || C < 1 || step < 0) return BSA_ERR_ARG;
+  if (!frames || !counts || !aligned(frames, 4) || !aligned(counts, 4)) return BSA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int threads = 128;
+  lvsa_build_index_kernel<<<(T + threads - 1) / threads, threads, 0, st>>>(T, T_per, C, step, frames, counts);
+  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  // over budget iff some t has |G_s u {t}| > C (pure function of the scalars)
+  const int s_mod = step % T_per;
+  const int nG = (s_mod < T) ? (T - 1 - s_mod) / T_per + 1 : 0;
+  const bool has_non_anchor = nG < T;
+  const bool over = (nG > C) || (has_non_anchor && nG + 1 > C);
+  return over ? BSA_WARN_OVER_BUDGET : BSA_OK;
+}
+
+size_t bsa_workspace_bytes(int op, int N, int H, int d, const bsa_index* index) {
+  if (N < 1 || H < 1 || (d != 64 && d != 128)) return static_cast<size_t>(-1);
+  if (op == BSA_OP_DENSE_BLOCKMASS) return 0;
+  if (op != BSA_OP_BLOCKSPARSE_FWD || !index) return static_cast<size_t>(-1);
+  if (index->kind == BSA_INDEX_BLOCKS) return 0;
+  if (index->kind != BSA_INDEX_LVSA_FRAMES || index->T < 1 || index->T > kMaxFrames || N % index->T)
+    return static_cast<size_t>(-1);
+  return lvsa_ws_layout(N, index->T).total;
+}
+
+int blocksparse_attn_fwd(const void* q, const void* k, const void* v, int N, int H, int d, float scale,
+                         const bsa_index* index, void* o, float* lse, void* workspace, size_t ws_bytes,
+                         void* stream) {
+  int rc = check_qkv(q, k, v, N, H, d, o, lse);
+  if (rc != BSA_OK) return rc;
+  if (!index || !std::isfinite(scale)) return BSA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams p = base_params(N, H, scale, o, lse);
+  const int nB = p.nB;
+  if (index->kind == BSA_INDEX_LVSA_FRAMES) {
+    const int T = index->T;
+    if (T < 1 || T > kMaxFrames) return BSA_ERR_ARG;
+    if (N % T) return BSA_ERR_SHAPE;
+    if (!index->frames || !index->counts) return BSA_ERR_ARG;
+    const LvsaWs w = lvsa_ws_layout(N, T);
+    if (!workspace || ws_bytes < w.total || !aligned(workspace, 256)) return BSA_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint32_t* fbits = reinterpret_cast<uint32_t*>(ws + w.fbits);
+    int32_t* tcnt = reinterpret_cast<int32_t*>(ws + w.cnt);
+    int32_t* tidx = reinterpret_cast<int32_t*>(ws + w.idx);
+    uint8_t* tflag = ws + w.flag;
+    lvsa_frame_bits_kernel<<<(T + 127) / 128, 128, 0, st>>>(T, index->frames, index->counts, fbits);
+    lvsa_tiles_kernel<<<(nB + 3) / 4, 128, 0, st>>>(N, T, N / T, nB, fbits, tcnt, tidx, tflag);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    p.list = tidx;
+    p.count = tcnt;
+    p.flags = tflag;
+    p.lhs = 0;
+    p.lrs = nB;
+    p.chs = 0;
+    p.fbits = fbits;
+    p.TW = (T + 31) / 32;
+    p.P = N / T;
+  } else if (index->kind == BSA_INDEX_BLOCKS) {
+    if (index->block != 128) return BSA_ERR_UNSUPPORTED;
+    if (index->H != H || index->nQB != nB || index->nKB != nB) return BSA_ERR_SHAPE;
+    if (!index->idx || !index->cnt) return BSA_ERR_ARG;
+    p.list = index->idx;
+    p.count = index->cnt;
+    p.flags = nullptr;
+    p.lhs = static_cast<long long>(index->nQB) * index->nKB;
+    p.lrs = index->nKB;
+    p.chs = index->nQB;
+  } else {
+    return BSA_ERR_ARG;
+  }
+  return launch_attn_any(d, false, q, k, v, N, H, p, st);
+}
+
+int attn_dense_blockmass(const void* q, const void* k, const void* v, int N, int H, int d, int block, float scale,
+                         void* o, float* lse, float* mass, void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  int rc = check_qkv(q, k, v, N, H, d, o, lse);
+  if (rc != BSA_OK) return rc;
+  if (!mass || !aligned(mass, 4) || !std::isfinite(scale)) return BSA_ERR_ARG;
+  if (block != 128) return BSA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams p = base_params(N, H, scale, o, lse);
+  p.dense = 1;
+  rc = launch_attn_any(d, false, q, k, v, N, H, p, st);
+  if (rc != BSA_OK) return rc;
+  p.mass = mass;
+  p.lse_in = lse;
+  return launch_attn_any(d, true, q, k, v, N, H, p, st);
+}
+
+int losa_select(const float* mass, int H, int nQB, int nKB, double tau, int32_t* idx, int32_t* cnt, void* stream) {
+  if (!mass || !idx || !cnt || !aligned(mass, 4) || !aligned(idx, 4) || !aligned(cnt, 4)) return BSA_ERR_ARG;
+  if (H < 1 || nQB < 1 || nKB < 1) return BSA_ERR_ARG;
+  if (nKB > kSelectMaxBlocks) return BSA_ERR_UNSUPPORTED;
+  if (!(tau > 0.0 && tau <= 1.0)) return BSA_ERR_ARG;
+  const long long rows = static_cast<long long>(H) * nQB;
+  if (rows > 0x7FFFFFFFLL) return BSA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = static_cast<size_t>(nKB) * 8;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(losa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSelectMaxBlocks * 8) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  losa_select_kernel<<<static_cast<unsigned>(rows), kSelectThreads, smem, st>>>(mass, nKB, tau, idx, cnt);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
+int bsa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BSA_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bsa_status, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_bsa_status, &zero, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"
+
+namespace {
+__global__ void debug_expired_wait_kernel(long long limit_ns) {
+  __shared__ alignas(8) unsigned long long bar;
+  if (threadIdx.x == 0) {
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    // nothing ever arrives on this barrier: the wait must give up by itself
+    mbar_wait(b, 0, limit_ns);
+  }
+}
+}  // namespace
+
+extern "C" int bsa_debug_expired_wait(long long limit_ns, void* stream) {
+  if (limit_ns < 100000LL || limit_ns > 10000000000LL) return BSA_ERR_ARG;
+  debug_expired_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}

@@ -30,8 +30,13 @@ from .lvsa import allowed_frames_matrix, dense_token_mask
 TILE = 128
 
 
-def kept_tiles(A: List[List[int]], T: int, N: int, tile: int = TILE) -> Tuple[List[List[int]], List[List[int]]]:
-    """Per query tile: ascending kept key tiles and their partial flags (0/1)."""
+def kept_tiles(A: List[List[int]], T: int, N: int, tile: int = TILE,
+               qtiles=None) -> Tuple[List[List[int]], List[List[int]]]:
+    """Per query tile: ascending kept key tiles and their partial flags (0/1).
+
+    ``qtiles`` (optional) restricts the evaluation to those query tiles; the
+    returned lists then follow that order.
+    """
     if N % T:
         raise ValueError("N must be a multiple of T")
     P = N // T
@@ -39,7 +44,7 @@ def kept_tiles(A: List[List[int]], T: int, N: int, tile: int = TILE) -> Tuple[Li
     nB = math.ceil(N / tile)
     idx: List[List[int]] = []
     flg: List[List[int]] = []
-    for qt in range(nB):
+    for qt in (range(nB) if qtiles is None else qtiles):
         q_lo, q_hi = qt * tile, min((qt + 1) * tile, N) - 1
         fq_lo, fq_hi = q_lo // P, q_hi // P
         row_i, row_f = [], []

@@ -1,0 +1,108 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side
+argument validation (no GPU work is enqueued by any call in this file)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsa.h")
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    from block_sparse_attention_lvsa_b200 import build
+    build.build()
+    from block_sparse_attention_lvsa_b200 import binding
+    return binding
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+\**([a-z_][a-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("lvsa_build_index", "attn_dense_blockmass", "losa_select", "blocksparse_attn_fwd"):
+        assert n in names
+
+
+def test_every_declared_symbol_exported(bsa):
+    lib = ctypes.CDLL(bsa.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(declared_functions()) <= set(bsa.EXPORTED)
+
+
+def test_status_strings(bsa):
+    assert bsa.status_string(0) == "BSA_OK"
+    assert bsa.status_string(-5) == "BSA_ERR_TIMEOUT"
+    assert bsa.status_string(12345) == "BSA_UNKNOWN_STATUS"
+
+
+def test_workspace_bytes(bsa):
+    ix = bsa.bsa_index()
+    ix.kind = bsa.BSA_INDEX_LVSA_FRAMES
+    ix.T = 126
+    n = bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 196560, 12, 128, ix)
+    nB = 1536
+    assert n >= nB * nB * 5 and n % 256 == 0
+    ix.kind = bsa.BSA_INDEX_BLOCKS
+    assert bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 32760, 40, 128, ix) == 0
+    assert bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, 32760, 40, 128, None) == 0
+    with pytest.raises(bsa.BsaError):
+        bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 100, 1, 128, None)
+    ix.kind = bsa.BSA_INDEX_LVSA_FRAMES
+    ix.T = 7
+    with pytest.raises(bsa.BsaError):      # T does not divide N
+        bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 100, 1, 128, ix)
+
+
+def test_host_validation_rejects_before_launch(bsa):
+    L = bsa.lib()
+    nul = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(0x10000)     # never dereferenced: rejected on the host first
+    assert L.lvsa_build_index(0, 4, 3, 4, 0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index(8, 0, 3, 4, 0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index(8, 4, 3, 4, -1, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index(8, 4, 3, 4, 0, nul, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index(2000, 4, 3, 4, 0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    ix = bsa.bsa_index()
+    ix.kind = bsa.BSA_INDEX_LVSA_FRAMES
+    ix.T = 8
+    ix.frames = ix.counts = 0x10000
+    f = L.blocksparse_attn_fwd
+    # unsupported head size
+    assert f(fake, fake, fake, 512, 2, 96, 0.1, ctypes.byref(ix), fake, fake, fake, 1 << 30, nul) == bsa.BSA_ERR_UNSUPPORTED
+    # null output
+    assert f(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(ix), nul, fake, fake, 1 << 30, nul) == bsa.BSA_ERR_ARG
+    # misaligned q
+    assert f(ctypes.c_void_p(0x10002), fake, fake, 512, 2, 64, 0.1, ctypes.byref(ix), fake, fake, fake, 1 << 30, nul) == bsa.BSA_ERR_ARG
+    # T does not divide N
+    assert f(fake, fake, fake, 500, 2, 64, 0.1, ctypes.byref(ix), fake, fake, fake, 1 << 30, nul) == bsa.BSA_ERR_SHAPE
+    # workspace too small
+    assert f(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(ix), fake, fake, fake, 16, nul) == bsa.BSA_ERR_WORKSPACE
+    # non-finite scale
+    assert f(fake, fake, fake, 512, 2, 64, float("nan"), ctypes.byref(ix), fake, fake, fake, 1 << 30, nul) == bsa.BSA_ERR_ARG
+    ix.kind = bsa.BSA_INDEX_BLOCKS
+    ix.block, ix.H, ix.nQB, ix.nKB = 64, 2, 4, 4
+    ix.idx = ix.cnt = 0x10000
+    assert f(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(ix), fake, fake, nul, 0, nul) == bsa.BSA_ERR_UNSUPPORTED
+    ix.block = 128
+    ix.nKB = 5
+    assert f(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(ix), fake, fake, nul, 0, nul) == bsa.BSA_ERR_SHAPE
+    ix.kind = 9
+    assert f(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(ix), fake, fake, nul, 0, nul) == bsa.BSA_ERR_ARG
+    g = L.attn_dense_blockmass
+    assert g(fake, fake, fake, 512, 2, 64, 64, 0.1, fake, fake, fake, nul, 0, nul) == bsa.BSA_ERR_UNSUPPORTED
+    assert g(fake, fake, fake, 512, 2, 64, 128, 0.1, fake, fake, nul, nul, 0, nul) == bsa.BSA_ERR_ARG
+    s = L.losa_select
+    assert s(fake, 2, 4, 4, 0.0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert s(fake, 2, 4, 4, 1.5, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert s(fake, 2, 4, 9000, 0.99, fake, fake, nul) == bsa.BSA_ERR_UNSUPPORTED
+    assert L.bsa_debug_expired_wait(10, nul) == bsa.BSA_ERR_ARG
