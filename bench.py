@@ -232,6 +232,9 @@ def run_b200(args, rank, world, local):
         raise SystemExit("bench.py needs a CUDA GPU (the product path has no CPU fallback)")
     peaks = load_peaks()
     wl = WORKLOADS[WORKLOAD]
+    if args.heads:
+        import dataclasses
+        wl = dataclasses.replace(wl, H=args.heads)      # profiling case only
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     N, H, d = wl.N, wl.H, wl.d
@@ -297,6 +300,12 @@ def run_b200(args, rank, world, local):
     value = job_flop / (max_total_ms / 1e3) / 1e12
     achieved = sum(flop_tile) / (sum(call_ms) / 1e3) / 1e12          # per-launch, this rank
     clocks = clk.summary()
+
+    if args.main_only:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "ms_per_call": statistics.median(call_ms),
+                              "tflops_kept_tiles": achieved, "heads": H, "profiling_case": True}), flush=True)
+        return
 
     # ---- dense run of the same kernel (every tile kept), same inputs
     dframes = torch.arange(wl.T, dtype=torch.int32, device=dev).repeat(wl.T, 1).contiguous()
@@ -453,6 +462,8 @@ def main():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--cpu-rows", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0, help="profiling only: override the head count")
+    ap.add_argument("--main-only", action="store_true", help="profiling only: timed LVSA steps, nothing else")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
