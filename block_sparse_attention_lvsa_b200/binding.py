@@ -35,7 +35,7 @@ BSA_OP_DENSE_BLOCKMASS = 2
 
 EXPORTED = ("lvsa_build_index", "attn_dense_blockmass", "losa_select", "blocksparse_attn_fwd",
             "bsa_workspace_bytes", "bsa_get_device_status", "bsa_status_string",
-            "bsa_debug_expired_wait", "bsa_version")
+            "bsa_debug_expired_wait", "bsa_version", "blocksparse_attn_fwd_noalloc")
 
 
 class BsaError(RuntimeError):
@@ -77,6 +77,7 @@ def _load():
         "bsa_status_string": (ctypes.c_char_p, [I]),
         "bsa_debug_expired_wait": (I, [ctypes.c_longlong, P]),
         "bsa_version": (ctypes.c_char_p, []),
+        "blocksparse_attn_fwd_noalloc": (I, [P, P, P, I, I, I, F, ctypes.POINTER(bsa_index), P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -187,6 +188,21 @@ def blocksparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, inde
     rc = _lib.blocksparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), N, H, d, float(scale), ctypes.byref(index),
                                    _ptr(o), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream))
     _check("blocksparse_attn_fwd", rc)
+    return o, lse
+
+
+def blocksparse_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, index: bsa_index,
+                                 o: torch.Tensor, lse: torch.Tensor, scale: Optional[float] = None,
+                                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """blocksparse_attn_fwd without a workspace: the library's static scratch array is
+    used instead, so the call allocates nothing (o and lse are the caller's)."""
+    _check_qkv(q, k, v)
+    N, H, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    rc = _lib.blocksparse_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), N, H, d, float(scale), ctypes.byref(index),
+                                           _ptr(o), _ptr(lse), _stream(stream))
+    _check("blocksparse_attn_fwd_noalloc", rc)
     return o, lse
 
 

@@ -287,3 +287,40 @@ extern "C" int bsa_debug_expired_wait(long long limit_ns, void* stream) {
   debug_expired_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// blocksparse_attn_fwd_noalloc: the workspace of blocksparse_attn_fwd placed in
+// a file-scope device array, for callers that cannot allocate device memory.
+// Host code must not use the array's name as a device address: the address
+// is looked up once per device with cudaGetSymbolAddress (that device
+// current) and passed on like a caller-owned workspace.
+namespace {
+constexpr size_t kNoAllocScratchBytes = BSA_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+}  // namespace
+
+extern "C" int blocksparse_attn_fwd_noalloc(const void* q, const void* k, const void* v, int N, int H, int d,
+                                            float scale, const bsa_index* index, void* o, float* lse,
+                                            void* stream) {
+  if (!index || N < 1) return BSA_ERR_ARG;
+  if (index->kind == BSA_INDEX_LVSA_FRAMES) {
+    if (index->T < 1 || index->T > kMaxFrames) return BSA_ERR_ARG;
+    if (N % index->T) return BSA_ERR_SHAPE;
+    if (lvsa_ws_layout(N, index->T).total > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return BSA_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return blocksparse_attn_fwd(q, k, v, N, H, d, scale, index, o, lse, scratch, kNoAllocScratchBytes, stream);
+}

@@ -198,6 +198,39 @@ int blocksparse_attn_fwd(const void* q, const void* k, const void* v,
                          const bsa_index* index, void* o, float* lse,
                          void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * blocksparse_attn_fwd_noalloc - the same computation as blocksparse_attn_fwd,
+ * for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for integration.
+ * Some callers cannot hand the library a workspace: plug-in hosts that own
+ * all device memory and give a plug-in no allocator, or latency-critical
+ * loops where a cudaMalloc (which may synchronise the device, or fail at run
+ * time) is not acceptable.  This entry point takes no workspace and
+ * allocates nothing: its scratch (the LVSA frame-pair bit matrix and key-tile
+ * lists) lives in one file-scope device array of BSA_NOALLOC_SCRATCH_BYTES
+ * bytes that every GPU loading the library holds until the process exits.
+ *
+ * Arguments, layouts and results are those of blocksparse_attn_fwd (both
+ * index kinds are accepted; block indexes need no scratch).  Returns
+ * BSA_ERR_WORKSPACE, before anything is enqueued, when an LVSA frame index
+ * needs more scratch than BSA_NOALLOC_SCRATCH_BYTES, i.e. when
+ * bsa_workspace_bytes(BSA_OP_BLOCKSPARSE_FWD, ...) exceeds it (up to about
+ * N = 234,000 tokens fits).
+ *
+ * The first call on a device looks up the device address of the array on
+ * that device (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture.  All calls on a device share the one
+ * array, and each call overwrites what the previous one left there before
+ * reading it (nothing has to start at zero).  Calls that overlap on the GPU
+ * (other streams, other host threads) race on the array: serialise them.
+ */
+#define BSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int blocksparse_attn_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 int N, int H, int d, float scale,
+                                 const bsa_index* index, void* o, float* lse,
+                                 void* stream);
+
 /* Operation codes for bsa_workspace_bytes. */
 enum {
   BSA_OP_BLOCKSPARSE_FWD = 1,
