@@ -8,24 +8,42 @@
 // Attention)" article, section "Balancing efficiency and quality" (one dense
 // step measuring exact inter-block mass, then the frozen block index).
 //
-// One CTA = one 128-row query tile of one head; it walks the key tiles its
-// list holds.  Warp roles (256 threads):
-//   warp 0      TMA producer: Q once, then K (and V) tiles into 2-deep rings
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 4..7  softmax warpgroup: thread r owns query row r (TMEM lane r)
-// TMEM columns: S0 [0,128) and S1 [128,256) (double-buffered scores, f32),
-// O [256, 256+d) (f32 accumulator).  S(j+1) = Q K(j+1)^T runs on the tensor
-// core while the softmax of tile j runs; then O += P(j) V(j), with P(j) in
-// shared memory (bf16, 128-byte swizzled, K-major).  The online softmax
-// keeps a running row maximum in log2 units and rescales O (TMEM ld/st)
-// only when the maximum grows by more than 2^8, which is exact after the
-// final division by the row sum.  Tiles flagged partial (frame boundary or
-// sequence end) get an element mask from the frame bit matrix.
+// One CTA = two neighbouring 128-row query tiles (0 = 2x, 1 = 2x+1) of one
+// head.  Every 128-key tile either of them keeps (the merge of their two
+// sorted lists) is loaded once by TMA and used by both, which halves the
+// bytes each SM pulls from L2 per FLOP.
+//
+// Warp roles (384 threads):
+//   warp 0       TMA producer: Q_0, Q_1 once, then K tiles (2-deep ring)
+//   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 2       TMA producer: V tiles (3-deep ring; forward only)
+//   warp 3       idle
+//   warps 4..7   softmax group 0: thread r owns row r of query tile 0
+//   warps 8..11  softmax group 1: thread r owns row r of query tile 1
+// TMEM columns: S_0 [0,128), S_1 [128,256) (f32 scores), O_0 [256,256+d),
+// O_1 [256+d, 256+2d) (f32 accumulators).  The softmax writes P (bf16, two
+// per 32-bit column) over the first 64 columns of its S tile and the PV
+// product reads it from there as the A operand (tcgen05.mma with A in
+// TMEM), so P never touches shared memory.
+//
+// Tensor-core order per key tile i (ping-pong between the two groups):
+//   S_0(i) = Q_0 K_i^T,  O_1 += P_1(i-1) V_{i-1},  S_1(i) = Q_1 K_i^T,
+//   O_0 += P_0(i) V_i
+// While group 0 turns S_0(i) into P_0(i) the tensor core runs O_1 and S_1,
+// and the other way round.  MMAs issued by one thread execute in order, so
+// S_x(i+1) (issued after O_x's PV) cannot overwrite P_x(i) before it is read,
+// and when a group sees S_x(i) complete, O_x is idle (its previous PV was
+// issued before S_x(i) and the completion barrier covers every earlier MMA):
+// the group rescales O_x in place when its running max grows by more than
+// 2^8 (exact after the final division).  Scores are read from TMEM twice
+// (row max, then exponentials), 64 columns at a time, to keep registers low.
+// Tiles flagged partial (frame boundary or sequence end) get an element mask
+// from the frame bit matrix.
 //
 // Mass mode (MASS = true) is the second pass of the dense measuring step:
-// it recomputes S tile by tile, forms p = exp2(s*scale*log2e - lse*log2e)
-// with the final row LSE of the forward pass and reduces p over the tile's
-// 128 x 128 entries into mass[h][qt][kt] (fixed reduction order).
+// it recomputes S, forms p = exp2(s*scale*log2e - lse*log2e) with the final
+// row LSE of the forward pass and reduces p over each 128 x 128 block into
+// mass[h][qt][kt] (fixed reduction order).
 #pragma once
 #include "ptx.cuh"
 
@@ -54,29 +72,46 @@ struct AttnParams {
   long long wait_limit_ns;
 };
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 384;
+constexpr int kQTilesPerCta = 2;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kKStages = 2;                        // K ring depth (128-key tiles)
+constexpr int kVStages = 3;                        // V ring depth (a V tile lives until O_1's PV)
 
 template <int D, bool MASS>
 struct AttnSmem {
-  static constexpr uint32_t kBox = 128 * 64 * 2;          // one 128-row x 64-col bf16 box
-  static constexpr uint32_t kTile = (D / 64) * kBox;       // 128 x D tile
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTile;               // 2 stages
-  static constexpr uint32_t kV = kK + 2 * kTile;           // 2 stages (fwd only)
-  static constexpr uint32_t kP = MASS ? kV : kV + 2 * kTile;   // 2 boxes (fwd only)
-  static constexpr uint32_t kBar = MASS ? kP : kP + 2 * kBox;
-  static constexpr uint32_t kNumBars = 20;
+  static constexpr uint32_t kBox = 128 * 128;               // 128 rows x 64 bf16 (128 B) per box
+  static constexpr uint32_t kTile = (D / 64) * kBox;        // one 128 x D tile
+  static constexpr uint32_t kQ = 0;                         // Q_0, Q_1
+  static constexpr uint32_t kK = kQ + 2 * kTile;
+  static constexpr uint32_t kV = kK + kKStages * kTile;
+  static constexpr uint32_t kBar = MASS ? kV : kV + kVStages * kTile;
+  static constexpr uint32_t kNumBars = 32;
   static constexpr uint32_t kHolder = kBar + kNumBars * 8;
-  static constexpr uint32_t kRed = kHolder + 16;           // 2 x 4 floats (mass reduction)
-  static constexpr uint32_t kBytes = kRed + 64;
-  static constexpr uint32_t kAlloc = kBytes + 1024;         // + alignment slack
-  static constexpr uint32_t kTmemCols = MASS ? 256 : 512;
+  static constexpr uint32_t kRed = kHolder + 16;            // [group][slot][warp] partial sums (mass)
+  static constexpr uint32_t kBytes = kRed + 2 * 2 * 4 * 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;          // + alignment slack
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmemO = 256;                    // O_0 at 256, O_1 at 256 + D
 };
 
 // barrier slots
-enum : int { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9,
-             B_SEMPTY = 11, B_PFULL = 13, B_PVDONE = 14, B_FINAL = 15, B_RFULL = 16, B_REMPTY = 18 };
+enum : int {
+  B_QFULL = 0,
+  B_KFULL = 1,                        // kKStages
+  B_KEMPTY = B_KFULL + kKStages,      // kKStages
+  B_VFULL = B_KEMPTY + kKStages,      // kVStages
+  B_VEMPTY = B_VFULL + kVStages,      // kVStages
+  B_SFULL = B_VEMPTY + kVStages,      // [group]
+  B_SEMPTY = B_SFULL + 2,             // [group] (mass mode)
+  B_PFULL = B_SEMPTY + 2,             // [group]
+  B_PVDONE = B_PFULL + 2,             // [group]
+  B_FINAL = B_PVDONE + 2,
+  B_RFULL = B_FINAL + 1,              // [group][slot]: 4
+  B_REMPTY = B_RFULL + 4,             // [group][slot]: 4
+  B_COUNT = B_REMPTY + 4
+};
+static_assert(B_COUNT <= 32, "barrier slots");
 
 __device__ __forceinline__ void set_bit_range(uint32_t (&mw)[4], int a, int b) {
 #pragma unroll
@@ -90,8 +125,8 @@ __device__ __forceinline__ void set_bit_range(uint32_t (&mw)[4], int a, int b) {
   }
 }
 
-// Element mask of one key tile for query frame fq: bit c set iff key k0+c < N
-// and frame(k0+c) is allowed for fq (all frames allowed when fbits is null).
+// Element mask of one 128-key tile for query frame fq: bit c set iff key
+// k0+c < N and frame(k0+c) is allowed for fq (all frames when fbits is null).
 __device__ __forceinline__ void tile_mask(const AttnParams& p, int fq, int k0, uint32_t (&mw)[4]) {
   mw[0] = mw[1] = mw[2] = mw[3] = 0u;
   const int kend = min(k0 + 128, p.N);
@@ -107,6 +142,68 @@ __device__ __forceinline__ void tile_mask(const AttnParams& p, int fq, int k0, u
   }
 }
 
+// Merge walk over the key-tile lists of the CTA's two query tiles.  Every
+// role runs its own copy over the same lists, so all of them see the same
+// sequence of (tile, in list 0, in list 1).  Entries outside [0, nB) are
+// skipped.
+struct PairLists {
+  const int32_t* l[2];
+  const uint8_t* f[2];
+  int n[2];
+  int dense, nB, N;
+  int i[2];
+
+  __device__ __forceinline__ int entry(int x) const {
+    return dense ? i[x] : __ldg(l[x] + i[x]);
+  }
+  // next kept tile: returns false at the end
+  __device__ __forceinline__ bool next(int& kt, bool (&in)[2], bool (&part)[2], bool& bad) {
+    while (true) {
+      int k[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        k[x] = (i[x] < n[x]) ? entry(x) : 0x7FFFFFFF;
+        if (k[x] != 0x7FFFFFFF && (k[x] < 0 || k[x] >= nB)) {   // out-of-range entry: skip
+          bad = true;
+          ++i[x];
+          k[x] = -1;
+        }
+      }
+      if (k[0] == -1 || k[1] == -1) continue;
+      if (k[0] == 0x7FFFFFFF && k[1] == 0x7FFFFFFF) return false;
+      kt = min(k[0], k[1]);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        in[x] = (k[x] == kt);
+        part[x] = false;
+        if (in[x]) {
+          part[x] = dense || f[x] == nullptr ? (kt * 128 + 128 > N) : (__ldg(f[x] + i[x]) != 0);
+          ++i[x];
+        }
+      }
+      return true;
+    }
+  }
+};
+
+__device__ __forceinline__ void apply_mask64(float (&s)[64], uint32_t m0, uint32_t m1) {
+#pragma unroll
+  for (int c = 0; c < 64; ++c)
+    if (!((((c < 32) ? m0 : m1) >> (c & 31)) & 1u)) s[c] = -INFINITY;
+}
+
+__device__ __forceinline__ float max64(const float (&s)[64]) {
+  float a = s[0], b = s[1], c = s[2], d = s[3];
+#pragma unroll
+  for (int j = 4; j < 64; j += 4) {
+    a = fmaxf(a, s[j]);
+    b = fmaxf(b, s[j + 1]);
+    c = fmaxf(c, s[j + 2]);
+    d = fmaxf(d, s[j + 3]);
+  }
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
 template <int D, bool MASS>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -120,47 +217,62 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile uint32_t* holder = reinterpret_cast<volatile uint32_t*>(gbase + L::kHolder);
 
-  const int qt = blockIdx.x, h = blockIdx.y;
+  const int qt0 = blockIdx.x * kQTilesPerCta, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long limit = p.wait_limit_ns;
 
-  // ---- this CTA's key-tile list
-  int n;
-  const int32_t* list = nullptr;
-  const uint8_t* flags = nullptr;
-  if (p.dense) {
-    n = p.nB;
-  } else {
-    n = p.count[static_cast<size_t>(h) * p.chs + qt];
-    if (n < 0 || n > p.lrs) {
-      if (threadIdx.x == 0) set_status(BSA_ERR_INDEX_RANGE);
-      n = n < 0 ? 0 : p.lrs;
+  // ---- the two query tiles' key-tile lists
+  PairLists pl;
+  pl.dense = p.dense;
+  pl.nB = p.nB;
+  pl.N = p.N;
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int qt = qt0 + x;
+    pl.l[x] = nullptr;
+    pl.f[x] = nullptr;
+    pl.i[x] = 0;
+    if (qt >= p.nB) {
+      pl.n[x] = 0;
+    } else if (p.dense) {
+      pl.n[x] = p.nB;
+    } else {
+      int n = p.count[static_cast<size_t>(h) * p.chs + qt];
+      if (n < 0 || n > p.lrs) {
+        if (threadIdx.x == 0) set_status(BSA_ERR_INDEX_RANGE);
+        n = n < 0 ? 0 : p.lrs;
+      }
+      pl.n[x] = n;
+      const size_t off = static_cast<size_t>(h) * p.lhs + static_cast<size_t>(qt) * p.lrs;
+      pl.l[x] = p.list + off;
+      if (p.flags) pl.f[x] = p.flags + off;
     }
-    const size_t off = static_cast<size_t>(h) * p.lhs + static_cast<size_t>(qt) * p.lrs;
-    list = p.list + off;
-    if (p.flags) flags = p.flags + off;
   }
-  auto tile_of = [&](int j) -> int { return p.dense ? j : __ldg(list + j); };
-  auto valid = [&](int kt) -> bool { return kt >= 0 && kt < p.nB; };
+  const bool active1 = (qt0 + 1) < p.nB;
+  const bool any_work = pl.n[0] > 0 || pl.n[1] > 0;
 
   // ---- setup: barriers (thread 0), TMEM (warp 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
       mbar_init(bar(B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
-      mbar_init(bar(B_SFULL + s), 1);
-      mbar_init(bar(B_SEMPTY + s), 128);
     }
-    mbar_init(bar(B_PFULL), 128);
-    mbar_init(bar(B_PVDONE), 1);
-    mbar_init(bar(B_FINAL), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(B_SFULL + x), 1);
+      mbar_init(bar(B_SEMPTY + x), 4);
+      mbar_init(bar(B_PFULL + x), 4);
+      mbar_init(bar(B_PVDONE + x), 1);
+    }
+    for (int s = 0; s < 4; ++s) {
       mbar_init(bar(B_RFULL + s), 4);
       mbar_init(bar(B_REMPTY + s), 1);
     }
+    mbar_init(bar(B_FINAL), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -176,111 +288,149 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
 
   if (warp == 0) {
-    // ================================================= TMA producer ====
-    if (lane == 0 && n > 0) {
+    // ============================================ TMA producer: Q, K ====
+    if (lane == 0 && any_work) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      if (!MASS) tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(bar(B_QFULL), L::kTile);
+      const int nq = active1 ? 2 : 1;
+      mbar_arrive_expect_tx(bar(B_QFULL), nq * L::kTile);
+      for (int x = 0; x < nq; ++x)
 #pragma unroll
-      for (int b = 0; b < D / 64; ++b)
-        tma_load_3d(base + L::kQ + b * L::kBox, &tmQ, bar(B_QFULL), b * 64, h, qt * 128);
-      int it = 0;
-      bool ok = true;
-      for (int j = 0; j < n && ok; ++j) {
-        const int kt = tile_of(j);
-        if (!valid(kt)) continue;
-        const int slot = it & 1;
-        if (it >= 2) ok = mbar_wait(bar(B_KEMPTY + slot), ((it - 2) >> 1) & 1, limit);
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(base + L::kQ + x * L::kTile + b * L::kBox, &tmQ, bar(B_QFULL), b * 64, h, (qt0 + x) * 128);
+      int it = 0, kt;
+      bool in[2], part[2], bad = false, ok = true;
+      while (ok && pl.next(kt, in, part, bad)) {
+        const int slot = it % kKStages;
+        if (it >= kKStages) ok = mbar_wait(bar(B_KEMPTY + slot), ((it - kKStages) / kKStages) & 1, limit);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(B_KFULL + slot), L::kTile);
 #pragma unroll
         for (int b = 0; b < D / 64; ++b)
-          tma_load_3d(base + L::kK + slot * L::kTile + b * L::kBox, &tmK, bar(B_KFULL + slot), b * 64, h,
-                      kt * 128);
-        if (!MASS) {
-          if (it >= 2) ok = mbar_wait(bar(B_VEMPTY + slot), ((it - 2) >> 1) & 1, limit);
-          if (!ok) break;
-          mbar_arrive_expect_tx(bar(B_VFULL + slot), L::kTile);
-#pragma unroll
-          for (int b = 0; b < D / 64; ++b)
-            tma_load_3d(base + L::kV + slot * L::kTile + b * L::kBox, &tmV, bar(B_VFULL + slot), b * 64, h,
-                        kt * 128);
-        }
+          tma_load_3d(base + L::kK + slot * L::kTile + b * L::kBox, &tmK, bar(B_KFULL + slot), b * 64, h, kt * 128);
         ++it;
       }
       // drain: wait (bounded) for this thread's own copies still in flight
       mbar_wait(bar(B_QFULL), 0, limit);
-      for (int u = max(0, it - 2); u < it; ++u) {
-        mbar_wait(bar(B_KFULL + (u & 1)), (u >> 1) & 1, limit);
-        if (!MASS) mbar_wait(bar(B_VFULL + (u & 1)), (u >> 1) & 1, limit);
+      for (int u = max(0, it - kKStages); u < it; ++u)
+        mbar_wait(bar(B_KFULL + u % kKStages), (u / kKStages) & 1, limit);
+    }
+  } else if (warp == 2) {
+    // ============================================== TMA producer: V ====
+    if (!MASS && lane == 0 && any_work) {
+      tma_prefetch_desc(&tmV);
+      int it = 0, kt;
+      bool in[2], part[2], bad = false, ok = true;
+      while (ok && pl.next(kt, in, part, bad)) {
+        const int slot = it % kVStages;
+        if (it >= kVStages) ok = mbar_wait(bar(B_VEMPTY + slot), ((it - kVStages) / kVStages) & 1, limit);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(B_VFULL + slot), L::kTile);
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_3d(base + L::kV + slot * L::kTile + b * L::kBox, &tmV, bar(B_VFULL + slot), b * 64, h, kt * 128);
+        ++it;
       }
+      for (int u = max(0, it - kVStages); u < it; ++u)
+        mbar_wait(bar(B_VFULL + u % kVStages), (u / kVStages) & 1, limit);
     }
   } else if (warp == 1) {
     // ================================================= MMA issuer ======
-    if (lane == 0 && n > 0) {
-      const uint32_t tS0 = tbase, tS1 = tbase + 128, tO = tbase + 256;
+    if (lane == 0 && any_work) {
       bool ok = true;
-      bool have_q = false;
-      int it = 0;
-      auto issue_pv = [&](int u) -> bool {
-        if (!mbar_wait(bar(B_PFULL), u & 1, limit)) return false;
-        if (!mbar_wait(bar(B_VFULL + (u & 1)), (u >> 1) & 1, limit)) return false;
-        tc_fence_after();
-        const uint32_t vbase = base + L::kV + (u & 1) * L::kTile;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {        // 16 keys per step
-          const uint64_t da = sw128_desc(base + L::kP + (kk >> 2) * L::kBox + (kk & 3) * 32, 16, 1024);
-          const uint64_t db = sw128_desc(vbase + kk * 2048, L::kBox, 1024);
-          mma_bf16_ss(tO, da, db, kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar(B_PVDONE));
-        tc_commit(bar(B_VEMPTY + (u & 1)));
-        return true;
-      };
-      for (int j = 0; j < n && ok; ++j) {
-        const int kt = tile_of(j);
-        if (!valid(kt)) continue;
-        if (!have_q) {
-          ok = mbar_wait(bar(B_QFULL), 0, limit);
-          have_q = true;
-          if (!ok) break;
-        }
-        const int b = it & 1;
-        if (it >= 2) ok = mbar_wait(bar(B_SEMPTY + b), ((it - 2) >> 1) & 1, limit);
-        if (!ok) break;
-        ok = mbar_wait(bar(B_KFULL + b), (it >> 1) & 1, limit);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kbase = base + L::kK + b * L::kTile;
-        const uint32_t dS = b ? tS1 : tS0;
+      const SmemDesc dQ[2] = {sw128_desc(base + L::kQ, 16, 1024), sw128_desc(base + L::kQ + L::kTile, 16, 1024)};
+      int cnt[2] = {0, 0};          // per query tile: key tiles processed
+      int it = 0, kt;
+      bool in[2], part[2], bad = false;
+      // O_1's PV of a key tile is issued during the next tile: remember it
+      int pend_it = -1, pend_c = 0;
+      bool pend_v_release = false;
+
+      auto qk = [&](int x, int ks) {
+        const SmemDesc dk = sw128_desc(base + L::kK + ks * L::kTile, 16, 1024);
+        const uint32_t dS = tbase + x * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {     // 16 channels per step
-          const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
-          const uint64_t da = sw128_desc(base + L::kQ + off, 16, 1024);
-          const uint64_t db = sw128_desc(kbase + off, 16, 1024);
-          mma_bf16_ss(dS, da, db, kIdescQK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(dS, dQ[x].lo + off, dQ[x].hi, dk.lo + off, dk.hi, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(B_SFULL + b));
-        tc_commit(bar(B_KEMPTY + b));
-        if (!MASS && it >= 1) ok = issue_pv(it - 1);
+        tc_commit(bar(B_SFULL + x));
+      };
+      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major)
+      auto pv = [&](int x, int vit, int c) -> bool {
+        if (!mbar_wait(bar(B_VFULL + vit % kVStages), (vit / kVStages) & 1, limit)) return false;
+        if (!mbar_wait(bar(B_PFULL + x), c & 1, limit)) return false;
+        tc_fence_after();
+        const SmemDesc dv = sw128_desc(base + L::kV + (vit % kVStages) * L::kTile, L::kBox, 1024);
+        const uint32_t tO = tbase + L::kTmemO + x * D;
+        const uint32_t tP = tbase + x * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)            // 16 keys per step: 8 TMEM columns of P, 2 KB of V
+          mma_bf16_ts(tO, tP + kk * 8, dv.lo + kk * 128, dv.hi, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(B_PVDONE + x));
+        return true;
+      };
+
+      if (!mbar_wait(bar(B_QFULL), 0, limit)) ok = false;
+      tc_fence_after();
+      while (ok && pl.next(kt, in, part, bad)) {
+        const int ks = it % kKStages;
+        ok = mbar_wait(bar(B_KFULL + ks), (it / kKStages) & 1, limit);
+        if (!ok) break;
+        tc_fence_after();
+        if (in[0]) {
+          if (MASS && cnt[0] > 0) ok = mbar_wait(bar(B_SEMPTY + 0), (cnt[0] - 1) & 1, limit);
+          if (!ok) break;
+          tc_fence_after();
+          qk(0, ks);
+        }
+        if (!MASS && pend_it >= 0) {
+          ok = pv(1, pend_it, pend_c);
+          if (!ok) break;
+          if (pend_v_release) tc_commit(bar(B_VEMPTY + pend_it % kVStages));
+          pend_it = -1;
+        }
+        if (in[1]) {
+          if (MASS && cnt[1] > 0) ok = mbar_wait(bar(B_SEMPTY + 1), (cnt[1] - 1) & 1, limit);
+          if (!ok) break;
+          tc_fence_after();
+          qk(1, ks);
+        }
+        tc_commit(bar(B_KEMPTY + ks));
+        if (!MASS) {
+          if (in[0]) {
+            ok = pv(0, it, cnt[0]);
+            if (!ok) break;
+            if (!in[1]) tc_commit(bar(B_VEMPTY + it % kVStages));
+          }
+          if (in[1]) {
+            pend_it = it;
+            pend_c = cnt[1];
+            pend_v_release = true;
+          }
+        }
+        if (in[0]) ++cnt[0];
+        if (in[1]) ++cnt[1];
         ++it;
       }
-      if (!MASS && ok && it >= 1) issue_pv(it - 1);
+      if (bad) set_status(BSA_ERR_INDEX_RANGE);
+      if (!MASS && ok && pend_it >= 0) {
+        if (pv(1, pend_it, pend_c)) tc_commit(bar(B_VEMPTY + pend_it % kVStages));
+      }
       // all issued MMAs complete before the CTA may release TMEM
       tc_commit(bar(B_FINAL));
       mbar_wait(bar(B_FINAL), 0, limit);
     }
   } else if (warp >= 4) {
-    // ================================================= softmax WG ======
-    const int r = threadIdx.x - 128;                 // row within tile = TMEM lane
+    // ================================================= softmax groups ==
+    const int x = (threadIdx.x - 128) >> 7;           // query tile 0 or 1 of this CTA
+    const int r = (threadIdx.x - 128) & 127;          // row within the tile = TMEM lane
+    const int qt = qt0 + x;
     const int q = qt * 128 + r;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const uint32_t tS0 = tbase + lane_off, tS1 = tbase + lane_off + 128;
-    const uint32_t tO = tbase + lane_off + 256;
+    const uint32_t tS = tbase + lane_off + x * 128;   // S_x; P_x over its first 64 columns
+    const uint32_t tO = tbase + lane_off + L::kTmemO + x * D;
     const int fq = (p.fbits != nullptr) ? (min(q, p.N - 1) / p.P) : 0;
-    const uint32_t pbase = base + L::kP + static_cast<uint32_t>(r) * 128;
-    const uint32_t rsw = static_cast<uint32_t>(r & 7);
 
     float m_run = -INFINITY, l_run = 0.f;
     float lse2 = 0.f;
@@ -288,117 +438,125 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const float v = (q < p.N) ? p.lse_in[static_cast<size_t>(h) * p.N + q] : -INFINITY;
       lse2 = isfinite(v) ? v * 1.4426950408889634f : INFINITY;   // rows without mass contribute 0
     }
-    float* red = reinterpret_cast<float*>(gbase + L::kRed);
+    float* red = reinterpret_cast<float*>(gbase + L::kRed) + x * 8;     // [slot][warp]
     bool ok = true;
-    int it = 0;
-    for (int j = 0; j < n && ok; ++j) {
-      const int kt = tile_of(j);
-      if (!valid(kt)) {
-        if (threadIdx.x == 128) set_status(BSA_ERR_INDEX_RANGE);
-        continue;
-      }
-      const int b = it & 1;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + b), (it >> 1) & 1, limit));
+    int cnt = 0;
+
+    int kt;
+    bool in[2], part[2], bad = false;
+    while (ok && pl.next(kt, in, part, bad)) {
+      if (!in[x]) continue;
+      uint32_t mw[4] = {0u, 0u, 0u, 0u};
+      if (part[x]) tile_mask(p, fq, kt * 128, mw);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + x), cnt & 1, limit));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld_x128(b ? tS1 : tS0, sr);
-      tc_fence_before();
-      mbar_arrive(bar(B_SEMPTY + b));
-      float* s = reinterpret_cast<float*>(sr);
-
-      const bool partial = p.dense ? (kt * 128 + 128 > p.N)
-                                   : (flags ? (flags[j] != 0) : (kt * 128 + 128 > p.N));
-      if (partial) {
-        uint32_t mw[4];
-        tile_mask(p, fq, kt * 128, mw);
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
-      }
 
       if (MASS) {
         float acc = 0.f;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) acc += ex2_approx(fmaf(s[c], p.sl2, -lse2));
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[64];
+          tmem_ld_x64(tS + 64 * half, sr);
+          float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
+          if (part[x]) apply_mask64(s, mw[2 * half], mw[2 * half + 1]);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) acc += ex2_approx(fmaf(s[c], p.sl2, -lse2));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_SEMPTY + x));
+        // reduce over the tile's rows and write mass[h][qt][kt] through a
+        // 2-slot ring guarded by mbarriers (no CTA-wide barrier in the loop)
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-        // hand the warp partial to row 0's thread through a 2-slot ring
-        // guarded by mbarriers (bounded waits; no CTA-wide barrier in the loop)
-        const int sl = it & 1;
+        const int sl = cnt & 1;
         bool okw = true;
         if (lane == 0) {
-          if (it >= 2) okw = mbar_wait(bar(B_REMPTY + sl), ((it - 2) >> 1) & 1, limit);
+          if (cnt >= 2) okw = mbar_wait(bar(B_REMPTY + 2 * x + sl), ((cnt - 2) >> 1) & 1, limit);
           if (okw) {
             red[sl * 4 + (warp & 3)] = acc;
-            mbar_arrive(bar(B_RFULL + sl));
+            mbar_arrive(bar(B_RFULL + 2 * x + sl));
           }
         }
         if (r == 0 && okw) {
-          okw = mbar_wait(bar(B_RFULL + sl), (it >> 1) & 1, limit);
+          okw = mbar_wait(bar(B_RFULL + 2 * x + sl), (cnt >> 1) & 1, limit);
           if (okw) {
             const volatile float* rr = red + sl * 4;
-            const float tot = (rr[0] + rr[1]) + (rr[2] + rr[3]);
-            p.mass[(static_cast<size_t>(h) * p.nB + qt) * p.nB + kt] = tot;
-            mbar_arrive(bar(B_REMPTY + sl));
+            p.mass[(static_cast<size_t>(h) * p.nB + qt) * p.nB + kt] = (rr[0] + rr[1]) + (rr[2] + rr[3]);
+            mbar_arrive(bar(B_REMPTY + 2 * x + sl));
           }
         }
         ok = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
         if (!ok) break;
       } else {
+        // pass 1: row max over the 128 scores
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[64];
+          tmem_ld_x64(tS + 64 * half, sr);
+          float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
+          if (part[x]) apply_mask64(s, mw[2 * half], mw[2 * half + 1]);
+          mx = fmaxf(mx, max64(s));
+        }
         const float mx2 = mx * p.sl2;
         const bool need = mx2 > m_run + kRescaleLog2;
         const float m_new = need ? mx2 : m_run;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          s[c] = ex2_approx(fmaf(s[c], p.sl2, -m_use));
-          rs += s[c];
-        }
         const float alpha = need ? ((m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new)) : 1.f;
-        l_run = l_run * alpha + rs;
-        m_run = m_new;
-        if (it > 0) {
-          // PV(it-1) must finish before O is rescaled and P is overwritten
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PVDONE), (it - 1) & 1, limit));
-          if (!ok) break;
-          tc_fence_after();
-          if (__any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+        // O_x is idle here (its last PV completed before S_x(i)): rescale in place
+        if (cnt > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t ov[32];
-              tmem_ld_x32(tO + c0, ov);
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t ov[32];
+            tmem_ld_x32(tO + c0, ov);
 #pragma unroll
-              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-              tmem_st_x32(tO + c0, ov);
-            }
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st_x32(tO + c0, ov);
           }
         }
-        // P (bf16) into the 128B-swizzled K-major operand tile: row r, 16B chunk c
+        // pass 2: p = exp2(s * scale * log2e - m), row sum, P (bf16) over S_x's first 64 columns
+        float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t addr = pbase + (c >> 3) * L::kBox + (((c & 7) ^ rsw) << 4);
-          st_shared_v4(addr, pack_bf16x2(s[8 * c + 0], s[8 * c + 1]), pack_bf16x2(s[8 * c + 2], s[8 * c + 3]),
-                       pack_bf16x2(s[8 * c + 4], s[8 * c + 5]), pack_bf16x2(s[8 * c + 6], s[8 * c + 7]));
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sr[64];
+          tmem_ld_x64(tS + 64 * half, sr);
+          float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
+          if (part[x]) apply_mask64(s, mw[2 * half], mw[2 * half + 1]);
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) {
+            const float e0 = ex2_approx(fmaf(s[c + 0], p.sl2, -m_use));
+            const float e1 = ex2_approx(fmaf(s[c + 1], p.sl2, -m_use));
+            const float e2 = ex2_approx(fmaf(s[c + 2], p.sl2, -m_use));
+            const float e3 = ex2_approx(fmaf(s[c + 3], p.sl2, -m_use));
+            rs0 += e0;
+            rs1 += e1;
+            rs2 += e2;
+            rs3 += e3;
+            pk[c / 2] = pack_bf16x2(e0, e1);
+            pk[c / 2 + 1] = pack_bf16x2(e2, e3);
+          }
+          tmem_st_x32(tS + 32 * half, pk);
         }
-        fence_proxy_async_smem();
+        l_run = l_run * alpha + ((rs0 + rs1) + (rs2 + rs3));
+        m_run = m_new;
         tc_fence_before();
-        mbar_arrive(bar(B_PFULL));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PFULL + x));
       }
-      ++it;
+      ++cnt;
     }
+    if (bad && r == 0) set_status(BSA_ERR_INDEX_RANGE);
 
     if (!MASS) {
-      // ---- epilogue: O / l (bf16) and LSE
-      if (ok && it > 0) {
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PVDONE), (it - 1) & 1, limit));
+      // ---- epilogue: O / l (bf16) and LSE for this group's query tile
+      if (ok && cnt > 0) {
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PVDONE + x), (cnt - 1) & 1, limit));
         tc_fence_after();
       }
-      const bool have = __all_sync(0xFFFFFFFFu, ok && it > 0);
+      const bool have = __all_sync(0xFFFFFFFFu, ok && cnt > 0);
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(q) * p.H + h) * D;
 #pragma unroll

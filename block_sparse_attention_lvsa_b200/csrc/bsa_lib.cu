@@ -39,13 +39,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D view (d, H, N) of a bf16 [N, H, d] tensor; box (64, 1, 128), 128B swizzle.
-bool make_qkv_map(CUtensorMap* m, const void* ptr, int N, int H, int d) {
+// 3-D view (d, H, N) of a bf16 [N, H, d] tensor; box (64, 1, rows), 128B swizzle.
+bool make_qkv_map(CUtensorMap* m, const void* ptr, int N, int H, int d, int rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -81,9 +81,11 @@ int launch_attn(const void* q, const void* k, const void* v, int N, int H, const
     attr_set[dev] = true;
   }
   CUtensorMap mq, mk, mv;
-  if (!make_qkv_map(&mq, q, N, H, D) || !make_qkv_map(&mk, k, N, H, D) || !make_qkv_map(&mv, v, N, H, D))
+  // query, key and value tiles are all 128 rows (boxes of 128 rows x 64 channels)
+  if (!make_qkv_map(&mq, q, N, H, D, 128) || !make_qkv_map(&mk, k, N, H, D, 128) ||
+      !make_qkv_map(&mv, v, N, H, D, 128))
     return BSA_ERR_CUDA;
-  dim3 grid(prm.nB, H);
+  dim3 grid((prm.nB + kQTilesPerCta - 1) / kQTilesPerCta, H);
   attn_tile_kernel<D, MASS><<<grid, kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
