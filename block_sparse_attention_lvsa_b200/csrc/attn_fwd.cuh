@@ -186,23 +186,52 @@ struct PairLists {
   }
 };
 
-__device__ __forceinline__ void apply_mask64(float (&s)[64], uint32_t m0, uint32_t m1) {
-#pragma unroll
-  for (int c = 0; c < 64; ++c)
-    if (!((((c < 32) ? m0 : m1) >> (c & 31)) & 1u)) s[c] = -INFINITY;
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
-__device__ __forceinline__ float max64(const float (&s)[64]) {
-  float a = s[0], b = s[1], c = s[2], d = s[3];
+__device__ __forceinline__ float max128(const float* s) {
+  float a = fmaxf(s[0], s[1]), b = fmaxf(s[2], s[3]), c = fmaxf(s[4], s[5]), d = fmaxf(s[6], s[7]);
 #pragma unroll
-  for (int j = 4; j < 64; j += 4) {
-    a = fmaxf(a, s[j]);
-    b = fmaxf(b, s[j + 1]);
-    c = fmaxf(c, s[j + 2]);
-    d = fmaxf(d, s[j + 3]);
+  for (int j = 8; j < 128; j += 8) {
+    a = fmax3(a, s[j], s[j + 1]);
+    b = fmax3(b, s[j + 2], s[j + 3]);
+    c = fmax3(c, s[j + 4], s[j + 5]);
+    d = fmax3(d, s[j + 6], s[j + 7]);
   }
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+  return fmax3(fmaxf(a, b), c, d);
 }
+
+__device__ __forceinline__ void apply_mask128(float* s, const uint32_t (&mw)[4]) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+}
+
+// 2^x on the FMA pipe, for x <= ~10 (inputs below -125 give ~2^-125, not 0;
+// the clamp keeps the exponent field of the result positive).
+// x = j + f with j = round(x) (adding and removing 1.5 * 2^23 rounds to the
+// nearest integer) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted
+// by Remez exchange for minimum relative error on [-1/2, 1/2] (max relative
+// error 7.5e-5, below the bf16 half-ulp of 2^-9 that P is rounded to); 2^j is
+// added to the exponent field as an integer.  Available to take part of the
+// exponentials of unmasked tiles off the MUFU unit (kPolyCols columns).
+__device__ __forceinline__ float exp2_poly3(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float j = t - 12582912.0f;
+  const float f = x - j;
+  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  // the exponent of t's bit pattern cancels: (0x4B400000 << 23) == 0 mod 2^32
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
+
+// columns of the 128 computed with exp2_poly3 in unmasked tiles (0: all on MUFU)
+constexpr int kPolyCols = 0;
 
 template <int D, bool MASS>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -454,14 +483,20 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
       if (MASS) {
         float acc = 0.f;
+        {
+          uint32_t sr[128];
+          tmem_ld_x128(tS, sr);
+          float* s = reinterpret_cast<float*>(sr);
+          if (part[x]) apply_mask128(s, mw);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sr[64];
-          tmem_ld_x64(tS + 64 * half, sr);
-          float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
-          if (part[x]) apply_mask64(s, mw[2 * half], mw[2 * half + 1]);
-#pragma unroll
-          for (int c = 0; c < 64; ++c) acc += ex2_approx(fmaf(s[c], p.sl2, -lse2));
+          for (int c = 0; c < 128; c += 4) {
+            a0 += ex2_approx(fmaf(s[c + 0], p.sl2, -lse2));
+            a1 += ex2_approx(fmaf(s[c + 1], p.sl2, -lse2));
+            a2 += ex2_approx(fmaf(s[c + 2], p.sl2, -lse2));
+            a3 += ex2_approx(fmaf(s[c + 3], p.sl2, -lse2));
+          }
+          acc = (a0 + a1) + (a2 + a3);
         }
         tc_fence_before();
         __syncwarp();
@@ -490,16 +525,12 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         ok = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
         if (!ok) break;
       } else {
-        // pass 1: row max over the 128 scores
-        float mx = -INFINITY;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sr[64];
-          tmem_ld_x64(tS + 64 * half, sr);
-          float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
-          if (part[x]) apply_mask64(s, mw[2 * half], mw[2 * half + 1]);
-          mx = fmaxf(mx, max64(s));
-        }
+        // one read of the 128 scores, then row max, exponentials, P in place
+        uint32_t sr[128];
+        tmem_ld_x128(tS, sr);
+        float* s = reinterpret_cast<float*>(sr);
+        if (part[x]) apply_mask128(s, mw);
+        const float mx = max128(s);
         const float mx2 = mx * p.sl2;
         const bool need = mx2 > m_run + kRescaleLog2;
         const float m_new = need ? mx2 : m_run;
@@ -516,30 +547,26 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tmem_st_x32(tO + c0, ov);
           }
         }
-        // pass 2: p = exp2(s * scale * log2e - m), row sum, P (bf16) over S_x's first 64 columns
+        // p = exp2(s * scale * log2e - m); P (bf16 pairs) packed in place into sr[0..63]
+        // (pair j overwrites sr[j] only after elements 2j, 2j+1 >= j are read)
         float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+        const bool poly = !part[x];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sr[64];
-          tmem_ld_x64(tS + 64 * half, sr);
-          float(&s)[64] = *reinterpret_cast<float(*)[64]>(sr);
-          if (part[x]) apply_mask64(s, mw[2 * half], mw[2 * half + 1]);
-          uint32_t pk[32];
+        for (int c = 0; c < 128; c += 4) {
+          float e[4];
 #pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const float e0 = ex2_approx(fmaf(s[c + 0], p.sl2, -m_use));
-            const float e1 = ex2_approx(fmaf(s[c + 1], p.sl2, -m_use));
-            const float e2 = ex2_approx(fmaf(s[c + 2], p.sl2, -m_use));
-            const float e3 = ex2_approx(fmaf(s[c + 3], p.sl2, -m_use));
-            rs0 += e0;
-            rs1 += e1;
-            rs2 += e2;
-            rs3 += e3;
-            pk[c / 2] = pack_bf16x2(e0, e1);
-            pk[c / 2 + 1] = pack_bf16x2(e2, e3);
+          for (int u = 0; u < 4; ++u) {
+            const float xx = fmaf(s[c + u], p.sl2, -m_use);
+            e[u] = (kPolyCols > 0 && poly && (c + u) < kPolyCols) ? exp2_poly3(xx) : ex2_approx(xx);
           }
-          tmem_st_x32(tS + 32 * half, pk);
+          rs0 += e[0];
+          rs1 += e[1];
+          rs2 += e[2];
+          rs3 += e[3];
+          sr[c / 2] = pack_bf16x2(e[0], e[1]);
+          sr[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
         }
+        tmem_st_x64(tS, sr);
         l_run = l_run * alpha + ((rs0 + rs1) + (rs2 + rs3));
         m_run = m_new;
         tc_fence_before();
