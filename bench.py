@@ -409,6 +409,30 @@ def run_e2e(bsa, wl, qkv, stream, frames, counts, ix, o, lse, ws, steps, kept_ti
             "ms_per_step": ms / steps, "steps": steps}
 
 
+def graph_timed(fn, n, reps=5):
+    """Median ms per call of `fn` captured `n` times into one CUDA graph (so the
+    host-side cost of each call is not part of the measurement)."""
+    fn()                                   # first call on the device does its set-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(n):
+                fn()
+    out = []
+    for i in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        if i:
+            out.append(a.elapsed_time(b) / n)
+    del g
+    return statistics.median(out)
+
+
 def run_losa(bsa, rank, stream, peaks):
     """LoSA on the Wan-2.1-14B shape: dense measuring step + mass, selection, frozen reuse."""
     wl = WORKLOADS["wan14b_losa"]
@@ -421,21 +445,25 @@ def run_losa(bsa, rank, stream, peaks):
     idx = torch.empty((H, nB, nB), dtype=torch.int32, device="cuda")
     cnt = torch.empty((H, nB), dtype=torch.int32, device="cuda")
 
-    def timed(fn, reps):
+    def timed(fn, reps, batch=1):
+        """Median ms per call; `batch` calls run back to back between the events
+        (for microsecond kernels, so host-side call overhead is not timed)."""
         out = []
         for i in range(reps + 1):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            fn()
+            for _ in range(batch):
+                fn()
             b.record(stream)
             torch.cuda.synchronize()
             if i:
-                out.append(a.elapsed_time(b))
+                out.append(a.elapsed_time(b) / batch)
         return statistics.median(out)
 
     t_dense = timed(lambda: bsa.attn_dense_blockmass(q, k, v, 128, wl.scale, o=o, lse=lse, mass=mass,
                                                      stream=stream), 3)
-    t_sel = timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt, stream=stream), 5)
+    # the selection runs in microseconds: time 50 launches replayed from a CUDA graph
+    t_sel = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 50)
     kept = int(cnt.sum().item())
     bix = bsa.block_index(idx, cnt)
     qs = [inputs.workload_qkv(wl, s, device="cuda") for s in (1, 2)]

@@ -102,9 +102,9 @@ enum : int {
   B_KEMPTY = B_KFULL + kKStages,      // kKStages
   B_VFULL = B_KEMPTY + kKStages,      // kVStages
   B_VEMPTY = B_VFULL + kVStages,      // kVStages
-  B_SFULL = B_VEMPTY + kVStages,      // [group]
-  B_SEMPTY = B_SFULL + 2,             // [group] (mass mode)
-  B_PFULL = B_SEMPTY + 2,             // [group]
+  B_SFULL = B_VEMPTY + kVStages,      // [group] (forward) / [group][buffer] (mass mode)
+  B_SEMPTY = B_SFULL + 4,             // [group][buffer] (mass mode)
+  B_PFULL = B_SEMPTY + 4,             // [group]
   B_PVDONE = B_PFULL + 2,             // [group]
   B_FINAL = B_PVDONE + 2,
   B_RFULL = B_FINAL + 1,              // [group][slot]: 4
@@ -291,9 +291,11 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
     }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_SEMPTY + s), 4);
+    }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(bar(B_SFULL + x), 1);
-      mbar_init(bar(B_SEMPTY + x), 4);
       mbar_init(bar(B_PFULL + x), 4);
       mbar_init(bar(B_PVDONE + x), 1);
     }
@@ -375,15 +377,17 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       int pend_it = -1, pend_c = 0;
       bool pend_v_release = false;
 
-      auto qk = [&](int x, int ks) {
+      // S = Q_x K^T into TMEM column block `sb` (forward: sb = x; mass mode:
+      // sb = 2x + buffer), completion signalled on SFULL + sb
+      auto qk = [&](int x, int sb, int ks) {
         const SmemDesc dk = sw128_desc(base + L::kK + ks * L::kTile, 16, 1024);
-        const uint32_t dS = tbase + x * 128;
+        const uint32_t dS = tbase + sb * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {     // 16 channels per step
           const uint32_t off = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
           mma_bf16_ss(dS, dQ[x].lo + off, dQ[x].hi, dk.lo + off, dk.hi, kIdescQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(B_SFULL + x));
+        tc_commit(bar(B_SFULL + sb));
       };
       // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major)
       auto pv = [&](int x, int vit, int c) -> bool {
@@ -408,10 +412,12 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (!ok) break;
         tc_fence_after();
         if (in[0]) {
-          if (MASS && cnt[0] > 0) ok = mbar_wait(bar(B_SEMPTY + 0), (cnt[0] - 1) & 1, limit);
+          // mass mode: S_0 double-buffered; the buffer is free once its scores were read
+          const int sb = MASS ? (cnt[0] & 1) : 0;
+          if (MASS && cnt[0] >= 2) ok = mbar_wait(bar(B_SEMPTY + sb), ((cnt[0] - 2) >> 1) & 1, limit);
           if (!ok) break;
           tc_fence_after();
-          qk(0, ks);
+          qk(0, sb, ks);
         }
         if (!MASS && pend_it >= 0) {
           ok = pv(1, pend_it, pend_c);
@@ -420,10 +426,11 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           pend_it = -1;
         }
         if (in[1]) {
-          if (MASS && cnt[1] > 0) ok = mbar_wait(bar(B_SEMPTY + 1), (cnt[1] - 1) & 1, limit);
+          const int sb = MASS ? (2 + (cnt[1] & 1)) : 1;
+          if (MASS && cnt[1] >= 2) ok = mbar_wait(bar(B_SEMPTY + sb), ((cnt[1] - 2) >> 1) & 1, limit);
           if (!ok) break;
           tc_fence_after();
-          qk(1, ks);
+          qk(1, sb, ks);
         }
         tc_commit(bar(B_KEMPTY + ks));
         if (!MASS) {
@@ -477,7 +484,9 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       if (!in[x]) continue;
       uint32_t mw[4] = {0u, 0u, 0u, 0u};
       if (part[x]) tile_mask(p, fq, kt * 128, mw);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + x), cnt & 1, limit));
+      // forward: one S buffer per group; mass mode: two, alternating
+      const int sb = MASS ? (2 * x + (cnt & 1)) : x;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + sb), MASS ? ((cnt >> 1) & 1) : (cnt & 1), limit));
       if (!ok) break;
       tc_fence_after();
 
@@ -485,7 +494,10 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         float acc = 0.f;
         {
           uint32_t sr[128];
-          tmem_ld_x128(tS, sr);
+          tmem_ld_x128(tbase + lane_off + sb * 128, sr);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_SEMPTY + sb));     // buffer free for the next QK^T
           float* s = reinterpret_cast<float*>(sr);
           if (part[x]) apply_mask128(s, mw);
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
@@ -498,9 +510,6 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
           acc = (a0 + a1) + (a2 + a3);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_SEMPTY + x));
         // reduce over the tile's rows and write mass[h][qt][kt] through a
         // 2-slot ring guarded by mbarriers (no CTA-wide barrier in the loop)
 #pragma unroll

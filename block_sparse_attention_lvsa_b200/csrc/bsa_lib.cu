@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "ptx.cuh"
@@ -247,17 +248,39 @@ int losa_select(const float* mass, int H, int nQB, int nKB, double tau, int32_t*
   const long long rows = static_cast<long long>(H) * nQB;
   if (rows > 0x7FFFFFFFLL) return BSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t smem = static_cast<size_t>(nKB) * 8;
+  // rows of up to 2048 blocks: keys in registers, 8 warps (one row each) per CTA
+  if (nKB <= 2048) {
+    const int wpc = 8;
+    const long long ctas = std::min<long long>((rows + wpc - 1) / wpc, 1LL << 20);
+    const dim3 grid(static_cast<unsigned>(ctas)), block(wpc * 32);
+    const int r = static_cast<int>(rows);
+    if (nKB <= 256)
+      losa_select_reg_kernel<8><<<grid, block, 0, st>>>(mass, r, nKB, tau, idx, cnt);
+    else if (nKB <= 512)
+      losa_select_reg_kernel<16><<<grid, block, 0, st>>>(mass, r, nKB, tau, idx, cnt);
+    else if (nKB <= 1024)
+      losa_select_reg_kernel<32><<<grid, block, 0, st>>>(mass, r, nKB, tau, idx, cnt);
+    else
+      losa_select_reg_kernel<64><<<grid, block, 0, st>>>(mass, r, nKB, tau, idx, cnt);
+    return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+  }
+  // longer rows: keys in shared memory, warps per CTA sized to <= 96 KB
+  const size_t row_bytes = static_cast<size_t>(nKB) * 8;
+  const int wpc = static_cast<int>(std::min<size_t>(8, std::max<size_t>(1, (96 * 1024) / row_bytes)));
+  const size_t smem = row_bytes * wpc;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(losa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSelectMaxBlocks * 8) != cudaSuccess)
+    // largest request: 96 KB (several warps) or one row of kSelectMaxBlocks keys (64 KB)
+    if (cudaFuncSetAttribute(losa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+        cudaSuccess)
       return BSA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  losa_select_kernel<<<static_cast<unsigned>(rows), kSelectThreads, smem, st>>>(mass, nKB, tau, idx, cnt);
+  const long long ctas = std::min<long long>((rows + wpc - 1) / wpc, 1LL << 20);
+  losa_select_kernel<<<static_cast<unsigned>(ctas), wpc * 32, smem, st>>>(mass, static_cast<int>(rows), nKB, tau,
+                                                                         idx, cnt);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
 
