@@ -363,9 +363,12 @@ def run_b200(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-# DRAM bytes per launch of the attention kernel from an ncu capture of this
-# workload (read + write); None until measured for the current kernel.
-TRAFFIC_PER_LAUNCH = None
+# DRAM bytes (read + write) per launch of the attention kernel at the full
+# 12-head workload: the ncu capture of the 4-head case of the same workload
+# (654.1 MB read + 192.3 MB written, step-0 index) scaled by 12/4 - traffic
+# grows with the number of heads.  Must be re-measured (or set to None)
+# whenever the kernel changes.
+TRAFFIC_PER_LAUNCH = 2.539e9
 
 
 def inputs_wl(wl, rank):
@@ -488,7 +491,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--cpu-rows", type=int, default=16384)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: override the head count")
     ap.add_argument("--main-only", action="store_true", help="profiling only: timed LVSA steps, nothing else")
