@@ -35,10 +35,10 @@
 // and when a group sees S_x(i) complete, O_x is idle (its previous PV was
 // issued before S_x(i) and the completion barrier covers every earlier MMA):
 // the group rescales O_x in place when its running max grows by more than
-// 2^8 (exact after the final division).  Scores are read from TMEM twice
-// (row max, then exponentials), 64 columns at a time, to keep registers low.
-// Tiles flagged partial (frame boundary or sequence end) get an element mask
-// from the frame bit matrix.
+// 2^8 (exact after the final division).  Each thread reads its row's 128
+// scores from TMEM once, takes the row max, then forms the exponentials and
+// packs P over the same registers.  Tiles flagged partial (frame boundary or
+// sequence end) get an element mask from the frame bit matrix.
 //
 // Mass mode (MASS = true) is the second pass of the dense measuring step:
 // it recomputes S, forms p = exp2(s*scale*log2e - lse*log2e) with the final
@@ -148,38 +148,42 @@ __device__ __forceinline__ void tile_mask(const AttnParams& p, int fq, int k0, u
 // skipped.
 struct PairLists {
   const int32_t* l[2];
-  const uint8_t* f[2];
   int n[2];
   int dense, nB, N;
   int i[2];
+  int cur[2];      // entry at i[x] (loaded one step ahead), 0x7FFFFFFF past the end
 
-  __device__ __forceinline__ int entry(int x) const {
-    return dense ? i[x] : __ldg(l[x] + i[x]);
+  __device__ __forceinline__ int load(int x, int j) const {
+    return (j < n[x]) ? (dense ? j : ld_pinned_s32(l[x] + j)) : 0x7FFFFFFF;
+  }
+  __device__ __forceinline__ void start() {
+    cur[0] = load(0, 0);
+    cur[1] = load(1, 0);
+  }
+  // advance list x; the next entry's load is issued now and used a call later
+  __device__ __forceinline__ void advance(int x) {
+    ++i[x];
+    cur[x] = load(x, i[x]);
   }
   // next kept tile: returns false at the end
-  __device__ __forceinline__ bool next(int& kt, bool (&in)[2], bool (&part)[2], bool& bad) {
+  __device__ __forceinline__ bool next(int& kt, bool (&in)[2], bool& bad) {
     while (true) {
-      int k[2];
+      bool skipped = false;
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        k[x] = (i[x] < n[x]) ? entry(x) : 0x7FFFFFFF;
-        if (k[x] != 0x7FFFFFFF && (k[x] < 0 || k[x] >= nB)) {   // out-of-range entry: skip
+        if (cur[x] != 0x7FFFFFFF && (cur[x] < 0 || cur[x] >= nB)) {   // out-of-range entry: skip
           bad = true;
-          ++i[x];
-          k[x] = -1;
+          advance(x);
+          skipped = true;
         }
       }
-      if (k[0] == -1 || k[1] == -1) continue;
-      if (k[0] == 0x7FFFFFFF && k[1] == 0x7FFFFFFF) return false;
-      kt = min(k[0], k[1]);
+      if (skipped) continue;
+      if (cur[0] == 0x7FFFFFFF && cur[1] == 0x7FFFFFFF) return false;
+      kt = min(cur[0], cur[1]);
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        in[x] = (k[x] == kt);
-        part[x] = false;
-        if (in[x]) {
-          part[x] = dense || f[x] == nullptr ? (kt * 128 + 128 > N) : (__ldg(f[x] + i[x]) != 0);
-          ++i[x];
-        }
+        in[x] = (cur[x] == kt);
+        if (in[x]) advance(x);
       }
       return true;
     }
@@ -252,6 +256,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   // ---- the two query tiles' key-tile lists
   PairLists pl;
+  const uint8_t* flg[2] = {nullptr, nullptr};     // per-entry partial flags (softmax only)
   pl.dense = p.dense;
   pl.nB = p.nB;
   pl.N = p.N;
@@ -259,7 +264,6 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   for (int x = 0; x < 2; ++x) {
     const int qt = qt0 + x;
     pl.l[x] = nullptr;
-    pl.f[x] = nullptr;
     pl.i[x] = 0;
     if (qt >= p.nB) {
       pl.n[x] = 0;
@@ -274,9 +278,10 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       pl.n[x] = n;
       const size_t off = static_cast<size_t>(h) * p.lhs + static_cast<size_t>(qt) * p.lrs;
       pl.l[x] = p.list + off;
-      if (p.flags) pl.f[x] = p.flags + off;
+      if (p.flags) flg[x] = p.flags + off;
     }
   }
+  pl.start();
   const bool active1 = (qt0 + 1) < p.nB;
   const bool any_work = pl.n[0] > 0 || pl.n[1] > 0;
 
@@ -330,8 +335,8 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int b = 0; b < D / 64; ++b)
           tma_load_3d(base + L::kQ + x * L::kTile + b * L::kBox, &tmQ, bar(B_QFULL), b * 64, h, (qt0 + x) * 128);
       int it = 0, kt;
-      bool in[2], part[2], bad = false, ok = true;
-      while (ok && pl.next(kt, in, part, bad)) {
+      bool in[2], bad = false, ok = true;
+      while (ok && pl.next(kt, in, bad)) {
         const int slot = it % kKStages;
         if (it >= kKStages) ok = mbar_wait(bar(B_KEMPTY + slot), ((it - kKStages) / kKStages) & 1, limit);
         if (!ok) break;
@@ -351,8 +356,8 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (!MASS && lane == 0 && any_work) {
       tma_prefetch_desc(&tmV);
       int it = 0, kt;
-      bool in[2], part[2], bad = false, ok = true;
-      while (ok && pl.next(kt, in, part, bad)) {
+      bool in[2], bad = false, ok = true;
+      while (ok && pl.next(kt, in, bad)) {
         const int slot = it % kVStages;
         if (it >= kVStages) ok = mbar_wait(bar(B_VEMPTY + slot), ((it - kVStages) / kVStages) & 1, limit);
         if (!ok) break;
@@ -368,14 +373,11 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else if (warp == 1) {
     // ================================================= MMA issuer ======
     if (lane == 0 && any_work) {
-      bool ok = true;
+      bool ok = true, bad = false;
       const SmemDesc dQ[2] = {sw128_desc(base + L::kQ, 16, 1024), sw128_desc(base + L::kQ + L::kTile, 16, 1024)};
       int cnt[2] = {0, 0};          // per query tile: key tiles processed
       int it = 0, kt;
-      bool in[2], part[2], bad = false;
-      // O_1's PV of a key tile is issued during the next tile: remember it
-      int pend_it = -1, pend_c = 0;
-      bool pend_v_release = false;
+      bool in[2];
 
       // S = Q_x K^T into TMEM column block `sb` (forward: sb = x; mass mode:
       // sb = 2x + buffer), completion signalled on SFULL + sb
@@ -389,11 +391,15 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         tc_commit(bar(B_SFULL + sb));
       };
-      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major)
-      auto pv = [&](int x, int vit, int c) -> bool {
+      // wait until V of key tile `vit` and P_x of the group's c-th tile are in place
+      auto pv_ready = [&](int x, int vit, int c) -> bool {
         if (!mbar_wait(bar(B_VFULL + vit % kVStages), (vit / kVStages) & 1, limit)) return false;
-        if (!mbar_wait(bar(B_PFULL + x), c & 1, limit)) return false;
+        if (!mbar_wait_spin(bar(B_PFULL + x), c & 1, limit)) return false;
         tc_fence_after();
+        return true;
+      };
+      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major)
+      auto pv = [&](int x, int vit, int c) {
         const SmemDesc dv = sw128_desc(base + L::kV + (vit % kVStages) * L::kTile, L::kBox, 1024);
         const uint32_t tO = tbase + L::kTmemO + x * D;
         const uint32_t tP = tbase + x * 128;
@@ -401,58 +407,90 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int kk = 0; kk < 8; ++kk)            // 16 keys per step: 8 TMEM columns of P, 2 KB of V
           mma_bf16_ts(tO, tP + kk * 8, dv.lo + kk * 128, dv.hi, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_PVDONE + x));
-        return true;
       };
 
       if (!mbar_wait(bar(B_QFULL), 0, limit)) ok = false;
       tc_fence_after();
-      while (ok && pl.next(kt, in, part, bad)) {
-        const int ks = it % kKStages;
-        ok = mbar_wait(bar(B_KFULL + ks), (it / kKStages) & 1, limit);
-        if (!ok) break;
-        tc_fence_after();
-        if (in[0]) {
-          // mass mode: S_0 double-buffered; the buffer is free once its scores were read
-          const int sb = MASS ? (cnt[0] & 1) : 0;
-          if (MASS && cnt[0] >= 2) ok = mbar_wait(bar(B_SEMPTY + sb), ((cnt[0] - 2) >> 1) & 1, limit);
+      if constexpr (MASS) {
+        while (ok && pl.next(kt, in, bad)) {
+          const int ks = it % kKStages;
+          ok = mbar_wait(bar(B_KFULL + ks), (it / kKStages) & 1, limit);
           if (!ok) break;
           tc_fence_after();
-          qk(0, sb, ks);
-        }
-        if (!MASS && pend_it >= 0) {
-          ok = pv(1, pend_it, pend_c);
-          if (!ok) break;
-          if (pend_v_release) tc_commit(bar(B_VEMPTY + pend_it % kVStages));
-          pend_it = -1;
-        }
-        if (in[1]) {
-          const int sb = MASS ? (2 + (cnt[1] & 1)) : 1;
-          if (MASS && cnt[1] >= 2) ok = mbar_wait(bar(B_SEMPTY + sb), ((cnt[1] - 2) >> 1) & 1, limit);
-          if (!ok) break;
-          tc_fence_after();
-          qk(1, sb, ks);
-        }
-        tc_commit(bar(B_KEMPTY + ks));
-        if (!MASS) {
-          if (in[0]) {
-            ok = pv(0, it, cnt[0]);
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (!in[x]) continue;
+            // S_x double-buffered; a buffer is free once its scores were read
+            const int sb = 2 * x + (cnt[x] & 1);
+            if (cnt[x] >= 2) ok = ok && mbar_wait(bar(B_SEMPTY + sb), ((cnt[x] - 2) >> 1) & 1, limit);
             if (!ok) break;
+            tc_fence_after();
+            qk(x, sb, ks);
+            ++cnt[x];
+          }
+          if (!ok) break;
+          tc_commit(bar(B_KEMPTY + ks));
+          ++it;
+        }
+      } else {
+        // Issue order per key tile i: O_1 += P_1(i-1) V, S_1(i), [next tile
+        // lookup and K wait], O_0 += P_0(i) V, S_0(i+1).  PV_0(i) and
+        // S_0(i+1) go out back to back: any memory-pipe instruction issued
+        // after queued MMAs (a list load, an mbarrier probe) waits for the
+        // tensor core to take them, so the bookkeeping is done while the
+        // queue still holds PV_1 and S_1.  In-order execution keeps S_x(i+1)
+        // behind PV_x(i), which reads P_x(i) from the same TMEM columns.
+        int pend_it = -1, pend_c = 0;       // O_1's PV of an earlier tile, not yet issued
+        bool have = ok && pl.next(kt, in, bad);
+        if (have) {
+          ok = mbar_wait(bar(B_KFULL), 0, limit);
+          tc_fence_after();
+          if (ok && in[0]) qk(0, 0, 0);
+        }
+        while (ok && have) {
+          const int ks = it % kKStages;
+          if (pend_it >= 0) {
+            ok = pv_ready(1, pend_it, pend_c);
+            if (!ok) break;
+            pv(1, pend_it, pend_c);
+            tc_commit(bar(B_VEMPTY + pend_it % kVStages));
+            pend_it = -1;
+          }
+          if (in[1]) qk(1, 1, ks);
+          tc_commit(bar(B_KEMPTY + ks));
+          int nkt = 0;
+          bool nin[2] = {false, false};
+          const bool nhave = pl.next(nkt, nin, bad);
+          if (nhave) {
+            ok = mbar_wait(bar(B_KFULL + (it + 1) % kKStages), ((it + 1) / kKStages) & 1, limit);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (in[0]) {
+            ok = pv_ready(0, it, cnt[0]);
+            if (!ok) break;
+            pv(0, it, cnt[0]);
             if (!in[1]) tc_commit(bar(B_VEMPTY + it % kVStages));
           }
+          if (nhave && nin[0]) qk(0, 0, (it + 1) % kKStages);
           if (in[1]) {
             pend_it = it;
             pend_c = cnt[1];
-            pend_v_release = true;
           }
+          if (in[0]) ++cnt[0];
+          if (in[1]) ++cnt[1];
+          ++it;
+          kt = nkt;
+          in[0] = nin[0];
+          in[1] = nin[1];
+          have = nhave;
         }
-        if (in[0]) ++cnt[0];
-        if (in[1]) ++cnt[1];
-        ++it;
+        if (ok && pend_it >= 0 && pv_ready(1, pend_it, pend_c)) {
+          pv(1, pend_it, pend_c);
+          tc_commit(bar(B_VEMPTY + pend_it % kVStages));
+        }
       }
       if (bad) set_status(BSA_ERR_INDEX_RANGE);
-      if (!MASS && ok && pend_it >= 0) {
-        if (pv(1, pend_it, pend_c)) tc_commit(bar(B_VEMPTY + pend_it % kVStages));
-      }
       // all issued MMAs complete before the CTA may release TMEM
       tc_commit(bar(B_FINAL));
       mbar_wait(bar(B_FINAL), 0, limit);
@@ -478,12 +516,30 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     bool ok = true;
     int cnt = 0;
 
-    int kt;
-    bool in[2], part[2], bad = false;
-    while (ok && pl.next(kt, in, part, bad)) {
-      if (!in[x]) continue;
+    // this group's tiles are its own list's in-range entries, in list order
+    // (the merge walk of the producers visits exactly those, in that order)
+    const int nx = x ? pl.n[1] : pl.n[0];
+    const int32_t* lx = x ? pl.l[1] : pl.l[0];
+    const uint8_t* fx = x ? flg[1] : flg[0];
+    bool bad = false;
+    const bool listed = !p.dense, flagged = !p.dense && fx != nullptr;
+    // entry j + 1 (tile and flag) is loaded while tile j is processed
+    int kt_next = (nx > 0) ? (listed ? ld_pinned_s32(lx) : 0) : 0;
+    uint32_t f_next = (nx > 0 && flagged) ? ld_pinned_u8(fx) : 0u;
+    for (int j = 0; ok && j < nx; ++j) {
+      const int kt = kt_next;
+      const uint32_t fl = f_next;
+      if (j + 1 < nx) {
+        kt_next = listed ? ld_pinned_s32(lx + j + 1) : (j + 1);
+        if (flagged) f_next = ld_pinned_u8(fx + j + 1);
+      }
+      if (kt < 0 || kt >= p.nB) {
+        bad = true;
+        continue;
+      }
+      const bool part = flagged ? (fl != 0u) : (kt * 128 + 128 > p.N);
       uint32_t mw[4] = {0u, 0u, 0u, 0u};
-      if (part[x]) tile_mask(p, fq, kt * 128, mw);
+      if (part) tile_mask(p, fq, kt * 128, mw);
       // forward: one S buffer per group; mass mode: two, alternating
       const int sb = MASS ? (2 * x + (cnt & 1)) : x;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + sb), MASS ? ((cnt >> 1) & 1) : (cnt & 1), limit));
@@ -499,7 +555,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(B_SEMPTY + sb));     // buffer free for the next QK^T
           float* s = reinterpret_cast<float*>(sr);
-          if (part[x]) apply_mask128(s, mw);
+          if (part) apply_mask128(s, mw);
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
           for (int c = 0; c < 128; c += 4) {
@@ -538,7 +594,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         uint32_t sr[128];
         tmem_ld_x128(tS, sr);
         float* s = reinterpret_cast<float*>(sr);
-        if (part[x]) apply_mask128(s, mw);
+        if (part) apply_mask128(s, mw);
         const float mx = max128(s);
         const float mx2 = mx * p.sl2;
         const bool need = mx2 > m_run + kRescaleLog2;
@@ -559,7 +615,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // p = exp2(s * scale * log2e - m); P (bf16 pairs) packed in place into sr[0..63]
         // (pair j overwrites sr[j] only after elements 2j, 2j+1 >= j are read)
         float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-        const bool poly = !part[x];
+        const bool poly = !part;
 #pragma unroll
         for (int c = 0; c < 128; c += 4) {
           float e[4];

@@ -72,7 +72,11 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, long 
   const uint64_t t0 = globaltimer_ns();
   const long long c0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // several probes per clock check keep the time from a phase completing
+    // to this thread seeing it short
+#pragma unroll 1
+    for (int k = 0; k < 16; ++k)
+      if (mbar_try_wait(bar, parity)) return true;
     const long long dt = static_cast<long long>(globaltimer_ns() - t0);
     const long long dc = clock64() - c0;
     if (dt > limit_ns || dc > 4 * limit_ns) {
@@ -84,6 +88,53 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, long 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, limit_ns);
+}
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Same bound as mbar_wait, but polls with the non-suspending test_wait: for
+// a single thread on the critical path that must react to the phase flip at
+// once (the MMA issuer waiting for P).
+__device__ __noinline__ bool mbar_wait_spin_slow(uint32_t bar, uint32_t parity, long long limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  const long long c0 = clock64();
+  while (true) {
+#pragma unroll 1
+    for (int k = 0; k < 64; ++k)
+      if (mbar_test_wait(bar, parity)) return true;
+    const long long dt = static_cast<long long>(globaltimer_ns() - t0);
+    const long long dc = clock64() - c0;
+    if (dt > limit_ns || dc > 4 * limit_ns) {
+      set_status(BSA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, long long limit_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_spin_slow(bar, parity, limit_ns);
+}
+
+// Read-only global loads kept where they are written: a prefetch issued one
+// step ahead must not be sunk to its use by the compiler (as an invariant
+// __ldg may be), or its latency lands on the critical path.
+__device__ __forceinline__ int32_t ld_pinned_s32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_pinned_u8(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
 }
 
 // ------------------------------------------------------------------ TMA --
