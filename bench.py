@@ -365,10 +365,10 @@ def run_b200(args, rank, world, local):
 
 # DRAM bytes (read + write) per launch of the attention kernel at the full
 # 12-head workload: the ncu capture of the 4-head case of the same workload
-# (654.1 MB read + 192.3 MB written, step-0 index) scaled by 12/4 - traffic
+# (672.6 MB read + 196.6 MB written, step-0 index) scaled by 12/4 - traffic
 # grows with the number of heads.  Must be re-measured (or set to None)
 # whenever the kernel changes.
-TRAFFIC_PER_LAUNCH = 2.539e9
+TRAFFIC_PER_LAUNCH = 2.607e9
 
 
 def inputs_wl(wl, rank):
@@ -485,6 +485,29 @@ def run_losa(bsa, rank, stream, peaks):
             "status": bsa.status_string(status)}
 
 
+def run_select_only():
+    """Profiling case for the LoSA selection alone, small on the device: block
+    masses from a 4-head dense measuring step on the Wan-2.1-14B shape, tiled
+    to that workload's 40 heads (10,240 rows of 256 key blocks)."""
+    import dataclasses
+    import block_sparse_attention_lvsa_b200.binding as bsa
+    wl = dataclasses.replace(WORKLOADS["wan14b_losa"], H=4)
+    q, k, v = inputs.workload_qkv(wl, 0, device="cuda")
+    _, _, mass4 = bsa.attn_dense_blockmass(q, k, v, 128, wl.scale)
+    del q, k, v
+    mass = mass4.repeat(10, 1, 1).contiguous()
+    idx, cnt = bsa.losa_select(mass, wl.tau)
+    for _ in range(3):
+        bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt)
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": "losa_select", "rows": mass.shape[0] * mass.shape[1], "nKB": mass.shape[2],
+                      "us": a.elapsed_time(b) * 1e3, "status": bsa.status_string(bsa.get_device_status())}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -495,7 +518,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: override the head count")
     ap.add_argument("--main-only", action="store_true", help="profiling only: timed LVSA steps, nothing else")
+    ap.add_argument("--select-only", action="store_true", help="profiling only: the LoSA selection, small case")
     args = ap.parse_args()
+    if args.select_only:
+        run_select_only()
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_init(args.gpus)

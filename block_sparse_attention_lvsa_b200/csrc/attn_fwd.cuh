@@ -197,15 +197,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 __device__ __forceinline__ float max128(const float* s) {
-  float a = fmaxf(s[0], s[1]), b = fmaxf(s[2], s[3]), c = fmaxf(s[4], s[5]), d = fmaxf(s[6], s[7]);
+  float a[8];
 #pragma unroll
-  for (int j = 8; j < 128; j += 8) {
-    a = fmax3(a, s[j], s[j + 1]);
-    b = fmax3(b, s[j + 2], s[j + 3]);
-    c = fmax3(c, s[j + 4], s[j + 5]);
-    d = fmax3(d, s[j + 6], s[j + 7]);
-  }
-  return fmax3(fmaxf(a, b), c, d);
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+  for (int j = 16; j < 128; j += 16)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[j + 2 * k], s[j + 2 * k + 1]);
+  return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
 }
 
 __device__ __forceinline__ void apply_mask128(float* s, const uint32_t (&mw)[4]) {
@@ -394,7 +393,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       // wait until V of key tile `vit` and P_x of the group's c-th tile are in place
       auto pv_ready = [&](int x, int vit, int c) -> bool {
         if (!mbar_wait(bar(B_VFULL + vit % kVStages), (vit / kVStages) & 1, limit)) return false;
-        if (!mbar_wait_spin(bar(B_PFULL + x), c & 1, limit)) return false;
+        if (!mbar_wait(bar(B_PFULL + x), c & 1, limit)) return false;
         tc_fence_after();
         return true;
       };
@@ -600,16 +599,19 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const bool need = mx2 > m_run + kRescaleLog2;
         const float m_new = need ? mx2 : m_run;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = need ? ((m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new)) : 1.f;
-        // O_x is idle here (its last PV completed before S_x(i)): rescale in place
-        if (cnt > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.f)) {
+        float alpha = 1.f;
+        if (__any_sync(0xFFFFFFFFu, need)) {
+          alpha = need ? ((m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new)) : 1.f;
+          // O_x is idle here (its last PV completed before S_x(i)): rescale in place
+          if (cnt > 0) {
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t ov[32];
-            tmem_ld_x32(tO + c0, ov);
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t ov[32];
+              tmem_ld_x32(tO + c0, ov);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-            tmem_st_x32(tO + c0, ov);
+              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+              tmem_st_x32(tO + c0, ov);
+            }
           }
         }
         // p = exp2(s * scale * log2e - m); P (bf16 pairs) packed in place into sr[0..63]

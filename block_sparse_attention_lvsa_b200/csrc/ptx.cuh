@@ -31,12 +31,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // ------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -64,63 +58,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with parity `parity` of barrier `bar` has completed.
-// Gives up after `limit_ns` nanoseconds of %globaltimer (or 4*limit_ns SM
-// clock cycles, in case the timer does not advance), records
-// BSA_ERR_TIMEOUT in the status word and returns false.  The first probe is
-// inlined; the bounded spin lives out of line.
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, long long limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
-  const long long c0 = clock64();
-  while (true) {
-    // several probes per clock check keep the time from a phase completing
-    // to this thread seeing it short
-#pragma unroll 1
-    for (int k = 0; k < 16; ++k)
-      if (mbar_try_wait(bar, parity)) return true;
-    const long long dt = static_cast<long long>(globaltimer_ns() - t0);
-    const long long dc = clock64() - c0;
-    if (dt > limit_ns || dc > 4 * limit_ns) {
-      set_status(BSA_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
+// Gives up after 2 * limit_ns SM clock cycles (limit_ns nanoseconds at
+// 2 GHz, longer at lower clocks), records BSA_ERR_TIMEOUT in the status
+// word and returns false.  The loop is inline and reads only clock64: an
+// out-of-line slow path or a %globaltimer read between probes measurably
+// delays the wake-up after the phase flips, and every handoff between the
+// TMA producer, the MMA issuer and the softmax warps pays that delay.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, limit_ns);
-}
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Same bound as mbar_wait, but polls with the non-suspending test_wait: for
-// a single thread on the critical path that must react to the phase flip at
-// once (the MMA issuer waiting for P).
-__device__ __noinline__ bool mbar_wait_spin_slow(uint32_t bar, uint32_t parity, long long limit_ns) {
-  const uint64_t t0 = globaltimer_ns();
   const long long c0 = clock64();
-  while (true) {
-#pragma unroll 1
-    for (int k = 0; k < 64; ++k)
-      if (mbar_test_wait(bar, parity)) return true;
-    const long long dt = static_cast<long long>(globaltimer_ns() - t0);
-    const long long dc = clock64() - c0;
-    if (dt > limit_ns || dc > 4 * limit_ns) {
+  const long long limit_cycles = 2 * limit_ns;
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - c0 > limit_cycles) {
       set_status(BSA_ERR_TIMEOUT);
       return false;
     }
   }
-}
-__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, long long limit_ns) {
-  if (mbar_test_wait(bar, parity)) return true;
-  return mbar_wait_spin_slow(bar, parity, limit_ns);
+  return true;
 }
 
 // Read-only global loads kept where they are written: a prefetch issued one

@@ -258,8 +258,9 @@ const char* bsa_status_string(int status);
 /*
  * bsa_debug_expired_wait - diagnostic for the bounded-wait machinery.
  * Enqueues one tiny kernel whose single thread waits on a barrier that
- * nothing ever signals, giving up after `limit_ns` nanoseconds (1e5..1e10)
- * and recording BSA_ERR_TIMEOUT in the status word.  Lets tests check that
+ * nothing ever signals, giving up after 2 * `limit_ns` SM clock cycles
+ * (`limit_ns` nanoseconds at 2 GHz; `limit_ns` in 1e5..1e10) and recording
+ * BSA_ERR_TIMEOUT in the status word.  Lets tests check that
  * an expired wait ends the kernel and leaves the context usable.  No part
  * of the pages corresponds to it.
  */
