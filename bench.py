@@ -447,6 +447,7 @@ def run_losa(bsa, rank, stream, peaks):
     mass = torch.empty((H, nB, nB), dtype=torch.float32, device="cuda")
     idx = torch.empty((H, nB, nB), dtype=torch.int32, device="cuda")
     cnt = torch.empty((H, nB), dtype=torch.int32, device="cuda")
+    ws = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, N, H, d), dtype=torch.uint8, device="cuda")
 
     def timed(fn, reps, batch=1):
         """Median ms per call; `batch` calls run back to back between the events
@@ -464,7 +465,7 @@ def run_losa(bsa, rank, stream, peaks):
         return statistics.median(out)
 
     t_dense = timed(lambda: bsa.attn_dense_blockmass(q, k, v, 128, wl.scale, o=o, lse=lse, mass=mass,
-                                                     stream=stream), 3)
+                                                     workspace=ws, stream=stream), 3)
     # the selection runs in microseconds: time 50 launches replayed from a CUDA graph
     t_sel = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 50)
     kept = int(cnt.sum().item())

@@ -207,8 +207,14 @@ def blocksparse_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
 
 
 def attn_dense_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int = 128,
-                         scale: Optional[float] = None, o=None, lse=None, mass=None, stream=None):
-    """Dense attention plus LoSA block mass; returns (o, lse, mass [H, nB, nB] f32)."""
+                         scale: Optional[float] = None, o=None, lse=None, mass=None,
+                         workspace: Optional[torch.Tensor] = None, stream=None):
+    """Dense attention plus LoSA block mass; returns (o, lse, mass [H, nB, nB] f32).
+
+    ``workspace`` (uint8 CUDA tensor, 256-byte aligned) holds at least one
+    head's log partial sums, nB * N * 4 bytes; more heads per pass when larger.
+    When omitted, ``workspace_bytes(BSA_OP_DENSE_BLOCKMASS, ...)`` bytes are allocated.
+    """
     _check_qkv(q, k, v)
     N, H, d = q.shape
     nB = math.ceil(N / 128)
@@ -220,8 +226,12 @@ def attn_dense_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bloc
         lse = torch.empty((H, N), dtype=torch.float32, device=q.device)
     if mass is None:
         mass = torch.empty((H, nB, nB), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(BSA_OP_DENSE_BLOCKMASS, N, H, d), dtype=torch.uint8,
+                                device=q.device)
     rc = _lib.attn_dense_blockmass(_ptr(q), _ptr(k), _ptr(v), N, H, d, block, float(scale),
-                                   _ptr(o), _ptr(lse), _ptr(mass), None, 0, _stream(stream))
+                                   _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel(),
+                                   _stream(stream))
     _check("attn_dense_blockmass", rc)
     return o, lse, mass
 

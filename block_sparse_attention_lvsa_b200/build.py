@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libbsa.so")
 SOURCES = ["bsa_lib.cu"]
-HEADERS = ["ptx.cuh", "lvsa_index.cuh", "losa_select.cuh", "attn_fwd.cuh"]
+HEADERS = ["ptx.cuh", "lvsa_index.cuh", "losa_select.cuh", "attn_fwd.cuh", "blockmass.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

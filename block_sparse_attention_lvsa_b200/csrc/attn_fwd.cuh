@@ -40,10 +40,13 @@
 // packs P over the same registers.  Tiles flagged partial (frame boundary or
 // sequence end) get an element mask from the frame bit matrix.
 //
-// Mass mode (MASS = true) is the second pass of the dense measuring step:
-// it recomputes S, forms p = exp2(s*scale*log2e - lse*log2e) with the final
-// row LSE of the forward pass and reduces p over each 128 x 128 block into
-// mass[h][qt][kt] (fixed reduction order).
+// Mass mode (MASS = true) is the dense measuring step of LoSA in one pass:
+// the same forward, which also writes, per query row and key tile, the log2
+// of that tile's share of the row's probability mass before normalisation,
+// lpart = log2(sum_k exp2(s_k * scale * log2e - m)) + m with the stabiliser m
+// the row used for the tile.  The block mass of a (query block, key block)
+// pair is then sum over the block's rows of exp2(lpart - lse * log2e), which
+// a separate reduction forms once the final LSE is known.
 #pragma once
 #include "ptx.cuh"
 
@@ -66,9 +69,9 @@ struct AttnParams {
   // outputs
   __nv_bfloat16* o;
   float* lse;
-  // mass pass
-  float* mass;
-  const float* lse_in;
+  // mass mode: lpart[(hl * nB + kt) * N + q] for local head hl = blockIdx.y
+  float* lpart;
+  int h_off;                        // head of blockIdx.y == 0
   long long wait_limit_ns;
 };
 
@@ -85,11 +88,10 @@ struct AttnSmem {
   static constexpr uint32_t kQ = 0;                         // Q_0, Q_1
   static constexpr uint32_t kK = kQ + 2 * kTile;
   static constexpr uint32_t kV = kK + kKStages * kTile;
-  static constexpr uint32_t kBar = MASS ? kV : kV + kVStages * kTile;
+  static constexpr uint32_t kBar = kV + kVStages * kTile;
   static constexpr uint32_t kNumBars = 32;
   static constexpr uint32_t kHolder = kBar + kNumBars * 8;
-  static constexpr uint32_t kRed = kHolder + 16;            // [group][slot][warp] partial sums (mass)
-  static constexpr uint32_t kBytes = kRed + 2 * 2 * 4 * 4;
+  static constexpr uint32_t kBytes = kHolder + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;          // + alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;                    // O_0 at 256, O_1 at 256 + D
@@ -102,14 +104,11 @@ enum : int {
   B_KEMPTY = B_KFULL + kKStages,      // kKStages
   B_VFULL = B_KEMPTY + kKStages,      // kVStages
   B_VEMPTY = B_VFULL + kVStages,      // kVStages
-  B_SFULL = B_VEMPTY + kVStages,      // [group] (forward) / [group][buffer] (mass mode)
-  B_SEMPTY = B_SFULL + 4,             // [group][buffer] (mass mode)
-  B_PFULL = B_SEMPTY + 4,             // [group]
+  B_SFULL = B_VEMPTY + kVStages,      // [group]
+  B_PFULL = B_SFULL + 2,              // [group]
   B_PVDONE = B_PFULL + 2,             // [group]
   B_FINAL = B_PVDONE + 2,
-  B_RFULL = B_FINAL + 1,              // [group][slot]: 4
-  B_REMPTY = B_RFULL + 4,             // [group][slot]: 4
-  B_COUNT = B_REMPTY + 4
+  B_COUNT = B_FINAL + 1
 };
 static_assert(B_COUNT <= 32, "barrier slots");
 
@@ -249,7 +248,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile uint32_t* holder = reinterpret_cast<volatile uint32_t*>(gbase + L::kHolder);
 
-  const int qt0 = blockIdx.x * kQTilesPerCta, h = blockIdx.y;
+  const int qt0 = blockIdx.x * kQTilesPerCta, h = blockIdx.y + p.h_off;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long limit = p.wait_limit_ns;
 
@@ -295,17 +294,10 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_init(bar(B_VFULL + s), 1);
       mbar_init(bar(B_VEMPTY + s), 1);
     }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(bar(B_SFULL + s), 1);
-      mbar_init(bar(B_SEMPTY + s), 4);
-    }
+    for (int x = 0; x < 2; ++x) mbar_init(bar(B_SFULL + x), 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(B_PFULL + x), 4);
       mbar_init(bar(B_PVDONE + x), 1);
-    }
-    for (int s = 0; s < 4; ++s) {
-      mbar_init(bar(B_RFULL + s), 4);
-      mbar_init(bar(B_REMPTY + s), 1);
     }
     mbar_init(bar(B_FINAL), 1);
     fence_mbar_init();
@@ -352,7 +344,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else if (warp == 2) {
     // ============================================== TMA producer: V ====
-    if (!MASS && lane == 0 && any_work) {
+    if (lane == 0 && any_work) {
       tma_prefetch_desc(&tmV);
       int it = 0, kt;
       bool in[2], bad = false, ok = true;
@@ -410,28 +402,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
       if (!mbar_wait(bar(B_QFULL), 0, limit)) ok = false;
       tc_fence_after();
-      if constexpr (MASS) {
-        while (ok && pl.next(kt, in, bad)) {
-          const int ks = it % kKStages;
-          ok = mbar_wait(bar(B_KFULL + ks), (it / kKStages) & 1, limit);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (!in[x]) continue;
-            // S_x double-buffered; a buffer is free once its scores were read
-            const int sb = 2 * x + (cnt[x] & 1);
-            if (cnt[x] >= 2) ok = ok && mbar_wait(bar(B_SEMPTY + sb), ((cnt[x] - 2) >> 1) & 1, limit);
-            if (!ok) break;
-            tc_fence_after();
-            qk(x, sb, ks);
-            ++cnt[x];
-          }
-          if (!ok) break;
-          tc_commit(bar(B_KEMPTY + ks));
-          ++it;
-        }
-      } else {
+      {
         // Issue order per key tile i: O_1 += P_1(i-1) V, S_1(i), [next tile
         // lookup and K wait], O_0 += P_0(i) V, S_0(i+1).  PV_0(i) and
         // S_0(i+1) go out back to back: any memory-pipe instruction issued
@@ -506,12 +477,6 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int fq = (p.fbits != nullptr) ? (min(q, p.N - 1) / p.P) : 0;
 
     float m_run = -INFINITY, l_run = 0.f;
-    float lse2 = 0.f;
-    if (MASS) {
-      const float v = (q < p.N) ? p.lse_in[static_cast<size_t>(h) * p.N + q] : -INFINITY;
-      lse2 = isfinite(v) ? v * 1.4426950408889634f : INFINITY;   // rows without mass contribute 0
-    }
-    float* red = reinterpret_cast<float*>(gbase + L::kRed) + x * 8;     // [slot][warp]
     bool ok = true;
     int cnt = 0;
 
@@ -539,56 +504,10 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const bool part = flagged ? (fl != 0u) : (kt * 128 + 128 > p.N);
       uint32_t mw[4] = {0u, 0u, 0u, 0u};
       if (part) tile_mask(p, fq, kt * 128, mw);
-      // forward: one S buffer per group; mass mode: two, alternating
-      const int sb = MASS ? (2 * x + (cnt & 1)) : x;
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + sb), MASS ? ((cnt >> 1) & 1) : (cnt & 1), limit));
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_SFULL + x), cnt & 1, limit));
       if (!ok) break;
       tc_fence_after();
-
-      if (MASS) {
-        float acc = 0.f;
-        {
-          uint32_t sr[128];
-          tmem_ld_x128(tbase + lane_off + sb * 128, sr);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_SEMPTY + sb));     // buffer free for the next QK^T
-          float* s = reinterpret_cast<float*>(sr);
-          if (part) apply_mask128(s, mw);
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-          for (int c = 0; c < 128; c += 4) {
-            a0 += ex2_approx(fmaf(s[c + 0], p.sl2, -lse2));
-            a1 += ex2_approx(fmaf(s[c + 1], p.sl2, -lse2));
-            a2 += ex2_approx(fmaf(s[c + 2], p.sl2, -lse2));
-            a3 += ex2_approx(fmaf(s[c + 3], p.sl2, -lse2));
-          }
-          acc = (a0 + a1) + (a2 + a3);
-        }
-        // reduce over the tile's rows and write mass[h][qt][kt] through a
-        // 2-slot ring guarded by mbarriers (no CTA-wide barrier in the loop)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-        const int sl = cnt & 1;
-        bool okw = true;
-        if (lane == 0) {
-          if (cnt >= 2) okw = mbar_wait(bar(B_REMPTY + 2 * x + sl), ((cnt - 2) >> 1) & 1, limit);
-          if (okw) {
-            red[sl * 4 + (warp & 3)] = acc;
-            mbar_arrive(bar(B_RFULL + 2 * x + sl));
-          }
-        }
-        if (r == 0 && okw) {
-          okw = mbar_wait(bar(B_RFULL + 2 * x + sl), (cnt >> 1) & 1, limit);
-          if (okw) {
-            const volatile float* rr = red + sl * 4;
-            p.mass[(static_cast<size_t>(h) * p.nB + qt) * p.nB + kt] = (rr[0] + rr[1]) + (rr[2] + rr[3]);
-            mbar_arrive(bar(B_REMPTY + 2 * x + sl));
-          }
-        }
-        ok = __shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0) != 0;
-        if (!ok) break;
-      } else {
+      {
         // one read of the 128 scores, then row max, exponentials, P in place
         uint32_t sr[128];
         tmem_ld_x128(tS, sr);
@@ -634,7 +553,14 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           sr[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
         }
         tmem_st_x64(tS, sr);
-        l_run = l_run * alpha + ((rs0 + rs1) + (rs2 + rs3));
+        const float rsum = (rs0 + rs1) + (rs2 + rs3);
+        if constexpr (MASS) {
+          // this tile's share of the row's mass, log2, before normalisation
+          if (q < p.N)
+            p.lpart[(static_cast<size_t>(blockIdx.y) * p.nB + kt) * p.N + q] =
+                (rsum > 0.f) ? (log2f(rsum) + m_use) : -INFINITY;
+        }
+        l_run = l_run * alpha + rsum;
         m_run = m_new;
         tc_fence_before();
         __syncwarp();
@@ -644,7 +570,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     if (bad && r == 0) set_status(BSA_ERR_INDEX_RANGE);
 
-    if (!MASS) {
+    {
       // ---- epilogue: O / l (bf16) and LSE for this group's query tile
       if (ok && cnt > 0) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PVDONE + x), (cnt - 1) & 1, limit));

@@ -15,6 +15,7 @@
 #include "lvsa_index.cuh"
 #include "losa_select.cuh"
 #include "attn_fwd.cuh"
+#include "blockmass.cuh"
 
 namespace {
 
@@ -68,8 +69,9 @@ int check_qkv(const void* q, const void* k, const void* v, int N, int H, int d, 
   return BSA_OK;
 }
 
+// grid over query-tile pairs x `grid_heads` heads, from head prm.h_off
 template <int D, bool MASS>
-int launch_attn(const void* q, const void* k, const void* v, int N, int H, const AttnParams& prm,
+int launch_attn(const void* q, const void* k, const void* v, int N, int H, int grid_heads, const AttnParams& prm,
                 cudaStream_t st) {
   using L = AttnSmem<D, MASS>;
   static bool attr_set[kMaxDevices] = {};
@@ -86,16 +88,17 @@ int launch_attn(const void* q, const void* k, const void* v, int N, int H, const
   if (!make_qkv_map(&mq, q, N, H, D, 128) || !make_qkv_map(&mk, k, N, H, D, 128) ||
       !make_qkv_map(&mv, v, N, H, D, 128))
     return BSA_ERR_CUDA;
-  dim3 grid((prm.nB + kQTilesPerCta - 1) / kQTilesPerCta, H);
+  dim3 grid((prm.nB + kQTilesPerCta - 1) / kQTilesPerCta, grid_heads);
   attn_tile_kernel<D, MASS><<<grid, kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
 
-int launch_attn_any(int d, bool mass, const void* q, const void* k, const void* v, int N, int H,
+int launch_attn_any(int d, bool mass, const void* q, const void* k, const void* v, int N, int H, int grid_heads,
                     const AttnParams& prm, cudaStream_t st) {
-  if (d == 128) return mass ? launch_attn<128, true>(q, k, v, N, H, prm, st)
-                            : launch_attn<128, false>(q, k, v, N, H, prm, st);
-  return mass ? launch_attn<64, true>(q, k, v, N, H, prm, st) : launch_attn<64, false>(q, k, v, N, H, prm, st);
+  if (d == 128) return mass ? launch_attn<128, true>(q, k, v, N, H, grid_heads, prm, st)
+                            : launch_attn<128, false>(q, k, v, N, H, grid_heads, prm, st);
+  return mass ? launch_attn<64, true>(q, k, v, N, H, grid_heads, prm, st)
+              : launch_attn<64, false>(q, k, v, N, H, grid_heads, prm, st);
 }
 
 AttnParams base_params(int N, int H, float scale, void* o, float* lse) {
@@ -110,6 +113,10 @@ AttnParams base_params(int N, int H, float scale, void* o, float* lse) {
   p.wait_limit_ns = kWaitLimitNs;
   return p;
 }
+
+// Workspace of the one-pass dense measuring step, per head: log2 partial
+// sums [nB key tiles][N rows] float32.
+size_t dense_mass_head_bytes(int N) { return static_cast<size_t>(n_tiles(N)) * static_cast<size_t>(N) * 4; }
 
 // Workspace layout for LVSA frame indexes.
 struct LvsaWs {
@@ -165,7 +172,12 @@ int lvsa_build_index(int T, int T_per, int W, int C, int step, int32_t* frames, 
 
 size_t bsa_workspace_bytes(int op, int N, int H, int d, const bsa_index* index) {
   if (N < 1 || H < 1 || (d != 64 && d != 128)) return static_cast<size_t>(-1);
-  if (op == BSA_OP_DENSE_BLOCKMASS) return 0;
+  if (op == BSA_OP_DENSE_BLOCKMASS) {
+    // every head in one pass, up to 4 GiB; any multiple of one head's share works
+    const size_t per_head = dense_mass_head_bytes(N);
+    const size_t heads = std::max<size_t>(1, std::min<size_t>(static_cast<size_t>(H), (size_t(4) << 30) / per_head));
+    return per_head * heads;
+  }
   if (op != BSA_OP_BLOCKSPARSE_FWD || !index) return static_cast<size_t>(-1);
   if (index->kind == BSA_INDEX_BLOCKS) return 0;
   if (index->kind != BSA_INDEX_LVSA_FRAMES || index->T < 1 || index->T > kMaxFrames || N % index->T)
@@ -219,25 +231,38 @@ int blocksparse_attn_fwd(const void* q, const void* k, const void* v, int N, int
   } else {
     return BSA_ERR_ARG;
   }
-  return launch_attn_any(d, false, q, k, v, N, H, p, st);
+  return launch_attn_any(d, false, q, k, v, N, H, H, p, st);
 }
 
 int attn_dense_blockmass(const void* q, const void* k, const void* v, int N, int H, int d, int block, float scale,
                          void* o, float* lse, float* mass, void* workspace, size_t ws_bytes, void* stream) {
-  (void)workspace;
-  (void)ws_bytes;
   int rc = check_qkv(q, k, v, N, H, d, o, lse);
   if (rc != BSA_OK) return rc;
   if (!mass || !aligned(mass, 4) || !std::isfinite(scale)) return BSA_ERR_ARG;
   if (block != 128) return BSA_ERR_UNSUPPORTED;
+  const size_t per_head = dense_mass_head_bytes(N);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < per_head) return BSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  AttnParams p = base_params(N, H, scale, o, lse);
-  p.dense = 1;
-  rc = launch_attn_any(d, false, q, k, v, N, H, p, st);
-  if (rc != BSA_OK) return rc;
-  p.mass = mass;
-  p.lse_in = lse;
-  return launch_attn_any(d, true, q, k, v, N, H, p, st);
+  const int nB = n_tiles(N);
+  // as many heads per pass as the workspace holds: the forward writes their
+  // log partial sums, the reduction turns them into block mass
+  const int hc = static_cast<int>(std::min<size_t>(static_cast<size_t>(H), ws_bytes / per_head));
+  for (int h0 = 0; h0 < H; h0 += hc) {
+    const int hn = std::min(hc, H - h0);
+    AttnParams p = base_params(N, H, scale, o, lse);
+    p.dense = 1;
+    p.lpart = static_cast<float*>(workspace);
+    p.h_off = h0;
+    rc = launch_attn_any(d, true, q, k, v, N, H, hn, p, st);
+    if (rc != BSA_OK) return rc;
+    const long long warps = static_cast<long long>(hn) * nB * nB;
+    const long long blocks = (warps + kMassThreads / 32 - 1) / (kMassThreads / 32);
+    if (blocks > 0x7FFFFFFFLL) return BSA_ERR_UNSUPPORTED;
+    blockmass_reduce_kernel<<<static_cast<unsigned>(blocks), kMassThreads, 0, st>>>(
+        static_cast<const float*>(workspace), lse, mass, N, nB, h0, hn);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
 }
 
 int losa_select(const float* mass, int H, int nQB, int nKB, double tau, int32_t* idx, int32_t* cnt, void* stream) {

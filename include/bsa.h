@@ -131,10 +131,19 @@ int lvsa_build_index(int T, int T_per, int W, int C, int step,
  * float32 softmax probabilities (not their bf16 rounding).  Sum over kb of
  * mass[h,qb,:] = number of tokens in qb.
  *
+ * One pass: the forward also writes, per head, key tile kt and row q, the
+ * log2 of the tile's share of the row's unnormalised mass (with the row's
+ * running stabiliser); a reduction then divides by the final row sum and
+ * adds the rows of each query block.  The probabilities are never
+ * recomputed.
+ *
  * q, k, v: in, bf16 [N,H,d].  block: must be 128.  scale: softmax scale
  * (normally d^-1/2).  o: out, bf16 [N,H,d].  lse: out, float32 [H,N].
  * mass: out, float32 [H][nB][nB], nB = ceil(N/128).
- * workspace, ws_bytes: unused for this call (pass NULL, 0); reserved.
+ * workspace, ws_bytes: device scratch, 256-byte aligned, owned by the
+ * caller, at least one head's share (nB * N * 4 bytes); heads are processed
+ * in passes of floor(ws_bytes / share) (bsa_workspace_bytes gives all heads
+ * in one pass up to 4 GiB).  Too small or misaligned: BSA_ERR_WORKSPACE.
  * Returns BSA_OK or a negative bsa_status.
  */
 int attn_dense_blockmass(const void* q, const void* k, const void* v,
@@ -239,7 +248,10 @@ enum {
 
 /*
  * bsa_workspace_bytes - scratch bytes the operation `op` needs for these
- * sizes (0 if none).  index may be NULL for BSA_OP_DENSE_BLOCKMASS.
+ * sizes (0 if none).  index may be NULL for BSA_OP_DENSE_BLOCKMASS.  For
+ * BSA_OP_DENSE_BLOCKMASS the answer is the share of as many heads as fit in
+ * 4 GiB (at least one, at most H), share = ceil(N/128) * N * 4 bytes; any
+ * workspace of at least one share is accepted by attn_dense_blockmass.
  * Returns (size_t)-1 for invalid arguments.
  */
 size_t bsa_workspace_bytes(int op, int N, int H, int d, const bsa_index* index);

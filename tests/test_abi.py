@@ -54,7 +54,11 @@ def test_workspace_bytes(bsa):
     assert n >= nB * nB * 5 and n % 256 == 0
     ix.kind = bsa.BSA_INDEX_BLOCKS
     assert bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 32760, 40, 128, ix) == 0
-    assert bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, 32760, 40, 128, None) == 0
+    share = 256 * 32760 * 4                        # key tiles x rows x float32, one head
+    assert bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, 32760, 40, 128, None) == 40 * share
+    share720 = 1772 * 226800 * 4                   # 720p: two heads fit in 4 GiB
+    assert bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, 226800, 40, 128, None) == 2 * share720
+    assert bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, 4 * 10 ** 6, 1, 128, None) == 31250 * 4 * 10 ** 6 * 4
     with pytest.raises(bsa.BsaError):
         bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 100, 1, 128, None)
     ix.kind = bsa.BSA_INDEX_LVSA_FRAMES
@@ -101,6 +105,9 @@ def test_host_validation_rejects_before_launch(bsa):
     g = L.attn_dense_blockmass
     assert g(fake, fake, fake, 512, 2, 64, 64, 0.1, fake, fake, fake, nul, 0, nul) == bsa.BSA_ERR_UNSUPPORTED
     assert g(fake, fake, fake, 512, 2, 64, 128, 0.1, fake, fake, nul, nul, 0, nul) == bsa.BSA_ERR_ARG
+    # the one-pass mass needs at least one head's share of workspace: 4 key tiles x 512 rows x 4 bytes
+    assert g(fake, fake, fake, 512, 2, 64, 128, 0.1, fake, fake, fake, nul, 0, nul) == bsa.BSA_ERR_WORKSPACE
+    assert g(fake, fake, fake, 512, 2, 64, 128, 0.1, fake, fake, fake, fake, 4 * 512 * 4 - 1, nul) == bsa.BSA_ERR_WORKSPACE
     s = L.losa_select
     assert s(fake, 2, 4, 4, 0.0, fake, fake, nul) == bsa.BSA_ERR_ARG
     assert s(fake, 2, 4, 4, 1.5, fake, fake, nul) == bsa.BSA_ERR_ARG

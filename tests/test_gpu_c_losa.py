@@ -46,6 +46,25 @@ def test_dense_blockmass_small(bsa, N, H, d):
             assert e <= gu.MASS_MAX, (h, qb, e)
 
 
+@pytest.mark.parametrize("N,H,d", [(1000, 3, 128), (300, 5, 64)])
+def test_dense_blockmass_head_passes(bsa, N, H, d):
+    """A workspace of one head's share (one pass per head) and of two shares
+    give the same o, lse and mass bit for bit as all heads in one pass."""
+    q, k, v = inputs.make_qkv(N, H, d, seed=7 * N + d, device="cuda")
+    share = (-(-N // 128)) * N * 4
+    full = bsa.attn_dense_blockmass(q, k, v, 128, d ** -0.5)
+    assert bsa.get_device_status() == bsa.BSA_OK
+    for shares in (1, 2):
+        ws = torch.empty(shares * share + 100, dtype=torch.uint8, device="cuda")
+        part = bsa.attn_dense_blockmass(q, k, v, 128, d ** -0.5, workspace=ws)
+        assert bsa.get_device_status() == bsa.BSA_OK
+        for a, b in zip(full, part):
+            assert torch.equal(a, b)
+    with pytest.raises(bsa.BsaError):
+        bsa.attn_dense_blockmass(q, k, v, 128, d ** -0.5,
+                                 workspace=torch.empty(share - 4, dtype=torch.uint8, device="cuda"))
+
+
 @pytest.fixture(scope="module")
 def losa_step0(bsa):
     """Dense measuring step on the 14B-shaped LoSA workload (full size)."""
