@@ -18,6 +18,8 @@ Readings taken where the page is open:
   * If |G_s u {t}| > C no set of size C holds every anchor and t; then
     A(t) = G_s u {t} and the call reports "over budget".  Anchors and t are
     never dropped.
+  * The other reading, "fixed window" (attended_frames_window): the window
+    holds W non-anchor frames, so |A(t)| = |G_s| + W and C plays no part.
 """
 from __future__ import annotations
 
@@ -57,6 +59,27 @@ def attended_frames(T: int, T_per: int, W: int, C: int, s: int) -> Tuple[List[Li
             dist += 1
         out.append(sorted(A))
     return out, over
+
+
+def attended_frames_window(T: int, T_per: int, W: int, s: int) -> List[List[int]]:
+    """A(t) under the fixed-window reading, ascending, for every query frame t.
+
+    [LVSA] sec. 2: A(t) = G u W(t).  Reading "fixed window" (the other
+    plain reading of the page, besides fill-to-budget): W(t) holds the W
+    non-anchor frames nearest to t - t itself first when it is not an
+    anchor, then by distance |f - t|, the earlier frame first at a tie - or
+    every non-anchor frame when there are fewer than W.  Hence
+    |A(t)| = |G_s| + min(W, T - |G_s|); t is always in A(t).
+    """
+    if T < 1 or T_per < 1 or W < 1 or s < 0:
+        raise ValueError("T, T_per, W must be >= 1 and s >= 0")
+    G = set(anchor_frames(T, T_per, s))
+    free = [f for f in range(T) if f not in G]
+    out: List[List[int]] = []
+    for t in range(T):
+        window = sorted(free, key=lambda f: (abs(f - t), f))[:W]
+        out.append(sorted(G | {t} | set(window)))
+    return out
 
 
 def allowed_frames_matrix(A: List[List[int]], T: int) -> np.ndarray:

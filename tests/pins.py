@@ -107,6 +107,69 @@ def check_lvsa_invariants(lvsa, T, T_per, W, C, steps):
         assert A == lvsa.attended_frames(T, T_per, W, C, s % T_per)[0]
 
 
+def read_lvsa_window_golden():
+    table = {}
+    with open(os.path.join(GOLDEN, "lvsa_window_T8_Tper4_W3.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, frames = line.split(":")
+            s, t = map(int, head.split())
+            table[(s, t)] = [int(x) for x in frames.split()]
+    return table
+
+
+def check_lvsa_window_golden(lvsa):
+    table = read_lvsa_window_golden()
+    assert len(table) == 32
+    for s in range(4):
+        A = lvsa.attended_frames_window(8, 4, 3, s)
+        for t in range(8):
+            assert A[t] == table[(s, t)], (s, t, A[t], table[(s, t)])
+
+
+def brute_force_window(T, T_per, W, s):
+    """Fixed-window reading by exhaustive search: among all sets X of
+    min(W, #non-anchors) non-anchor frames that hold t when t is not an
+    anchor, the one whose sorted (|f - t|, f) tuple is smallest."""
+    G = {f for f in range(T) if (f - s) % T_per == 0}
+    free = [f for f in range(T) if f not in G]
+    n = min(W, len(free))
+    out = []
+    for t in range(T):
+        best = None
+        for X in itertools.combinations(free, n):
+            if t not in G and t not in X:
+                continue
+            key = sorted((abs(f - t), f) for f in X)
+            if best is None or key < best[0]:
+                best = (key, X)
+        out.append(sorted(G | {t} | set(best[1])))
+    return out
+
+
+def check_lvsa_window_bruteforce(lvsa, T=8):
+    for T_per in (1, 2, 3, 4, 5, 9):
+        for W in (1, 2, 3, 5, 8):
+            for s in range(T_per + 1):
+                assert lvsa.attended_frames_window(T, T_per, W, s) == brute_force_window(T, T_per, W, s), \
+                    (T_per, W, s)
+
+
+def check_lvsa_window_invariants(lvsa, T, T_per, W, steps):
+    for s in steps:
+        G = {f for f in range(T) if (f - s) % T_per == 0}
+        A = lvsa.attended_frames_window(T, T_per, W, s)
+        for t in range(T):
+            a = A[t]
+            assert a == sorted(set(a)) and all(0 <= f < T for f in a)
+            assert G <= set(a) and t in a
+            assert len(a) == len(G) + min(W, T - len(G))
+        # the two readings agree once the budget is |G_s| + W (balanced configurations)
+        assert A == lvsa.attended_frames(T, T_per, W, min(T, len(G) + W), s)[0]
+
+
 # ---------------------------------------------------------------- tiles ---
 def random_allowed(T, rng, density=0.4):
     A = []

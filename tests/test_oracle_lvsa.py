@@ -63,3 +63,16 @@ def test_pair_count_closed_form():
         A, _ = lvsa.attended_frames(8, 4, 3, 4, s)
         m = lvsa.dense_token_mask(A, 64, 512)
         assert tiles.exact_pair_count(A, 8, 512) == int(m.sum())
+
+
+def test_window_golden_hand_derived_T8():
+    pins.check_lvsa_window_golden(lvsa)
+
+
+def test_window_bruteforce_T8():
+    pins.check_lvsa_window_bruteforce(lvsa)
+
+
+@pytest.mark.parametrize("T,T_per,W", [(8, 4, 3), (21, 5, 7), (126, 6, 15), (126, 21, 15), (63, 6, 15), (5, 9, 7)])
+def test_window_invariants(T, T_per, W):
+    pins.check_lvsa_window_invariants(lvsa, T, T_per, W, range(min(T_per, 8) + 1))

@@ -82,6 +82,35 @@ def test_lvsa_tiebreak_caught():
     assert fails(pins.check_lvsa_bruteforce, m)
 
 
+def mutant_lvsa_window(kind):
+    """Fixed-window reading with one planted mistake."""
+    m = clone(lvsa)
+
+    def window(T, T_per, W, s):
+        G = set(lvsa.anchor_frames(T, T_per, s))
+        free = [f for f in range(T) if f not in G]
+        out = []
+        for t in range(T):
+            if kind == "tie":            # later frame first at equal distance
+                order = sorted(free, key=lambda f: (abs(f - t), -f))
+            else:
+                order = sorted(free, key=lambda f: (abs(f - t), f))
+            if kind == "no_t":           # t not counted in its own window
+                order = [f for f in order if f != t]
+            n = W - 1 if kind == "short" else W
+            out.append(sorted(G | {t} | set(order[:n])))
+        return out
+    m.attended_frames_window = window
+    return m
+
+
+@pytest.mark.parametrize("kind", ["tie", "no_t", "short"])
+def test_lvsa_window_mistakes_caught(kind):
+    m = mutant_lvsa_window(kind)
+    assert fails(pins.check_lvsa_window_golden, m)
+    assert fails(pins.check_lvsa_window_bruteforce, m)
+
+
 def test_tiles_partial_flag_caught():
     m = clone(tiles)
 
