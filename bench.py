@@ -323,6 +323,9 @@ def run_b200(args, rank, world, local):
     dense_ms = statistics.median(dense_ms)
     dense_flop = 4 * d * H * nB * nB * 128 * 128
 
+    # ---- balanced variant of the same shape (T_per = 21: |A(t)| = C = 21 for every t and s)
+    balanced = run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws) if rank == 0 else None
+
     # ---- e2e: host buffers through the public API, copies inside the timed region
     e2e = run_e2e(bsa, wl, pool[0], stream, frames, counts, ix, o, lse, ws, max(2, min(args.steps, 5)),
                   kept_tiles, world)
@@ -353,6 +356,7 @@ def run_b200(args, rank, world, local):
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
         "losa": losa,
+        "balanced_tper21": balanced,
     }
     if rank == 0 and not args.no_cpu_baseline:
         dt, fl, n, cores = oracle_sample(wl, 0, args.cpu_rows, head=0, qkv=None, seed=7)
@@ -369,6 +373,33 @@ def run_b200(args, rank, world, local):
 # grows with the number of heads.  Must be re-measured (or set to None)
 # whenever the kernel changes.
 TRAFFIC_PER_LAUNCH = 2.607e9
+
+
+def run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws, calls=6):
+    """The balanced reading of the 6x-horizon shape (T_per = 21, 6 anchors +
+    15 window frames = C): ms per call and TFLOP/s on kept tiles over the
+    first `calls` steps (anchor phases 0..calls-1), each on its own inputs."""
+    wl = WORKLOADS["wan1.3b_6x_tper21"]
+    ms, flop, kept = [], 0, 0
+    for s in range(calls + 1):
+        bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, s, frames, counts, stream=stream)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        bsa.blocksparse_attn_fwd(*pool[s % len(pool)], ix, scale=wl.scale, o=o, lse=lse, workspace=ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if s == 0:
+            continue                                  # warm-up for this index shape
+        _, tcnt, _, _ = bsa.lvsa_workspace_views(ws, wl.N, wl.T)
+        k = int(tcnt.sum().item())
+        kept += k
+        flop += 4 * wl.d * wl.H * k * 128 * 128
+        ms.append(a.elapsed_time(b))
+    status = bsa.get_device_status()
+    nB = math.ceil(wl.N / 128)
+    return {"workload": "wan1.3b_6x_tper21: as the headline shape with T_per=21 (|A(t)| = C = 21 for every t, s)",
+            "ms_per_call": statistics.median(ms), "tflops_kept_tiles": flop / (sum(ms) / 1e3) / 1e12,
+            "kept_tile_fraction": kept / calls / (nB * nB), "steps": calls, "status": bsa.status_string(status)}
 
 
 def inputs_wl(wl, rank):

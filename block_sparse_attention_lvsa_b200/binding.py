@@ -33,7 +33,7 @@ BSA_INDEX_BLOCKS = 2
 BSA_OP_BLOCKSPARSE_FWD = 1
 BSA_OP_DENSE_BLOCKMASS = 2
 
-EXPORTED = ("lvsa_build_index", "attn_dense_blockmass", "losa_select", "blocksparse_attn_fwd",
+EXPORTED = ("lvsa_build_index", "lvsa_build_index_window", "attn_dense_blockmass", "losa_select", "blocksparse_attn_fwd",
             "bsa_workspace_bytes", "bsa_get_device_status", "bsa_status_string",
             "bsa_debug_expired_wait", "bsa_version", "blocksparse_attn_fwd_noalloc")
 
@@ -69,6 +69,7 @@ def _load():
     P, I, D, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float, ctypes.c_size_t
     sig = {
         "lvsa_build_index": (I, [I, I, I, I, I, P, P, P]),
+        "lvsa_build_index_window": (I, [I, I, I, I, P, P, P]),
         "attn_dense_blockmass": (I, [P, P, P, I, I, I, I, F, P, P, P, P, SZ, P]),
         "losa_select": (I, [P, I, I, I, D, P, P, P]),
         "blocksparse_attn_fwd": (I, [P, P, P, I, I, I, F, ctypes.POINTER(bsa_index), P, P, P, SZ, P]),
@@ -140,6 +141,20 @@ def lvsa_build_index(T: int, T_per: int, W: int, C: int, step: int,
     rc = _lib.lvsa_build_index(T, T_per, W, C, step, _ptr(frames), _ptr(counts), _stream(stream))
     _check("lvsa_build_index", rc, (BSA_OK, BSA_WARN_OVER_BUDGET))
     return frames, counts, rc == BSA_WARN_OVER_BUDGET
+
+
+def lvsa_build_index_window(T: int, T_per: int, W: int, step: int,
+                            frames: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
+                            device=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """A(t) under the fixed-window reading (W non-anchor frames): (frames [T,T] int32, counts [T] int32)."""
+    dev = device if device is not None else (frames.device if frames is not None else "cuda")
+    if frames is None:
+        frames = torch.empty((T, T), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty((T,), dtype=torch.int32, device=dev)
+    rc = _lib.lvsa_build_index_window(T, T_per, W, step, _ptr(frames), _ptr(counts), _stream(stream))
+    _check("lvsa_build_index_window", rc)
+    return frames, counts
 
 
 def lvsa_index(T: int, frames: torch.Tensor, counts: torch.Tensor) -> bsa_index:

@@ -170,6 +170,16 @@ int lvsa_build_index(int T, int T_per, int W, int C, int step, int32_t* frames, 
   return over ? BSA_WARN_OVER_BUDGET : BSA_OK;
 }
 
+int lvsa_build_index_window(int T, int T_per, int W, int step, int32_t* frames, int32_t* counts, void* stream) {
+  if (T < 1 || T > kMaxFrames || T_per < 1 || W < 1 || step < 0) return BSA_ERR_ARG;
+  // |G_s| = number of f in [0, T) with f = step mod T_per (mod T_per)
+  const int s_mod = step % T_per;
+  const int nG = (s_mod < T) ? (T - 1 - s_mod) / T_per + 1 : 0;
+  const int C = static_cast<int>(std::min<long long>(T, static_cast<long long>(nG) + W));
+  // |G_s u {t}| <= min(T, nG + 1) <= C, so the fill never reports over budget
+  return lvsa_build_index(T, T_per, W, C, step, frames, counts, stream);
+}
+
 size_t bsa_workspace_bytes(int op, int N, int H, int d, const bsa_index* index) {
   if (N < 1 || H < 1 || (d != 64 && d != 128)) return static_cast<size_t>(-1);
   if (op == BSA_OP_DENSE_BLOCKMASS) {

@@ -119,6 +119,26 @@ int lvsa_build_index(int T, int T_per, int W, int C, int step,
                      int32_t* frames, int32_t* counts, void* stream);
 
 /*
+ * lvsa_build_index_window - LVSA attended-frame sets under the fixed-window
+ * reading of the same passage.
+ *
+ * Source: [LVSA] section 2 (A(t) = G u W(t) with a local window of size W).
+ * Where lvsa_build_index fills each set to the budget C, this call reads
+ * the window as holding W non-anchor frames: W(t) = the W non-anchor frames
+ * nearest to t (t itself first when it is not an anchor, then by distance
+ * |f - t|, the earlier frame first at a tie, clipped to [0, T)), or every
+ * non-anchor frame when there are fewer; A(t) = G_s u {t} u W(t), so
+ * |A(t)| = |G_s| + min(W, T - |G_s|).  The sets equal lvsa_build_index's
+ * with C = min(T, |G_s| + W), which is how they are computed.
+ *
+ * frames, counts: as for lvsa_build_index.
+ * Limits: 1 <= T <= 1024, T_per >= 1, W >= 1, step >= 0.
+ * Returns BSA_OK, or BSA_ERR_ARG / BSA_ERR_CUDA.
+ */
+int lvsa_build_index_window(int T, int T_per, int W, int step,
+                            int32_t* frames, int32_t* counts, void* stream);
+
+/*
  * attn_dense_blockmass - dense attention forward that also emits LoSA block mass.
  *
  * Source: [LoSA] section "Balancing efficiency and quality" (one dense

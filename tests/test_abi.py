@@ -76,6 +76,10 @@ def test_host_validation_rejects_before_launch(bsa):
     assert L.lvsa_build_index(8, 4, 3, 4, -1, fake, fake, nul) == bsa.BSA_ERR_ARG
     assert L.lvsa_build_index(8, 4, 3, 4, 0, nul, fake, nul) == bsa.BSA_ERR_ARG
     assert L.lvsa_build_index(2000, 4, 3, 4, 0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index_window(0, 4, 3, 0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index_window(8, 4, 0, 0, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index_window(8, 4, 3, -1, fake, fake, nul) == bsa.BSA_ERR_ARG
+    assert L.lvsa_build_index_window(8, 4, 3, 0, fake, nul, nul) == bsa.BSA_ERR_ARG
     ix = bsa.bsa_index()
     ix.kind = bsa.BSA_INDEX_LVSA_FRAMES
     ix.T = 8

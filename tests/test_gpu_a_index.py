@@ -50,6 +50,34 @@ def test_build_index_random(bsa):
     check_index(bsa, 1, 1, 1, 1, 0)         # degenerate single frame
 
 
+def check_window_index(bsa, T, T_per, W, s):
+    frames, counts = bsa.lvsa_build_index_window(T, T_per, W, s, device="cuda")
+    A = olvsa.attended_frames_window(T, T_per, W, s)
+    fr = frames.cpu().numpy()
+    ct = counts.cpu().numpy()
+    for t in range(T):
+        assert ct[t] == len(A[t]), (T, T_per, W, s, t)
+        assert list(fr[t, :ct[t]]) == A[t], (T, T_per, W, s, t)
+        assert np.all(fr[t, ct[t]:] == -1)
+
+
+@pytest.mark.parametrize("name", LVSA_WL)
+def test_window_index_workloads(bsa, name):
+    """Fixed-window reading, bit-exact vs the oracle, every anchor phase."""
+    wl = WORKLOADS[name]
+    for s in sorted(set(list(range(wl.T_per + 1)) + [wl.steps - 1])):
+        check_window_index(bsa, wl.T, wl.T_per, wl.W, s)
+
+
+def test_window_index_random(bsa):
+    rng = np.random.default_rng(1)
+    for _ in range(60):
+        T = int(rng.integers(1, 300))
+        check_window_index(bsa, T, int(rng.integers(1, 40)), int(rng.integers(1, T + 3)), int(rng.integers(0, 100)))
+    check_window_index(bsa, 1024, 7, 30, 5)
+    check_window_index(bsa, 1, 1, 1, 0)
+
+
 def tile_lists(bsa, T, P, A, d=64):
     """Run the forward once (H=1) and decode the tile lists from the workspace."""
     N = T * P

@@ -159,5 +159,20 @@ def test_wan_6x_balanced(bsa):
     sampled_lvsa(bsa, WORKLOADS["wan1.3b_6x_tper21"], 2, 128, [3], 40)
 
 
+@pytest.mark.parametrize("name,s", [("wan1.3b_1x_c11", 0), ("wan1.3b_1x_c11", 3), ("wan1.3b_6x", 1)])
+def test_window_reading(bsa, name, s):
+    """Attention on the fixed-window frame sets (|A(t)| = |G_s| + W)."""
+    wl = WORKLOADS[name]
+    q, k, v = inputs.workload_qkv(wl, s, device="cuda")
+    frames, counts = bsa.lvsa_build_index_window(wl.T, wl.T_per, wl.W, s, device="cuda")
+    o, lse = bsa.blocksparse_attn_fwd(q, k, v, bsa.lvsa_index(wl.T, frames, counts), scale=wl.scale)
+    assert bsa.get_device_status() == bsa.BSA_OK
+    A = olvsa.attended_frames_window(wl.T, wl.T_per, wl.W, s)
+    rows = inputs.sample_rows(wl.N, wl.P, 128, 60 + s).numpy()
+    keys, group = gu.lvsa_keys(A, wl.P, wl.N)
+    Os, Ls = gu.oracle_rows(q, k, v, wl.scale, rows, [0, 5], keys, group)
+    gu.compare_rows(o, lse, Os, Ls, rows, f"{name} window s={s}")
+
+
 def test_720p_lvsa_full_size(bsa):
     sampled_lvsa(bsa, WORKLOADS["720p_14b"], 0, 128, [0, 39], 50)
