@@ -216,12 +216,14 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def config_block(wl, world):
+def config_block(wl, world, shard="replicas", H_total=None):
+    H_all = wl.H if H_total is None else H_total
     return {"workload": f"{wl.name}: LVSA block-sparse self-attention, Wan-2.1-1.3B shape at 6x horizon, "
-                        f"T={wl.T} frames x P={wl.P} tokens (N={wl.N}), H={wl.H}, d={wl.d}, "
+                        f"T={wl.T} frames x P={wl.P} tokens (N={wl.N}), H={H_all}, d={wl.d}, "
                         f"C={wl.C}, W={wl.W}, T_per={wl.T_per}, anchors rotated per step, fresh q/k/v per step",
-            "N": wl.N, "H": wl.H, "d": wl.d, "T": wl.T, "P": wl.P, "C": wl.C, "W": wl.W, "T_per": wl.T_per,
-            "global_batch": world, "seq_len": wl.N, "parallelism": f"replicas x{world}",
+            "N": wl.N, "H": H_all, "d": wl.d, "T": wl.T, "P": wl.P, "C": wl.C, "W": wl.W, "T_per": wl.T_per,
+            "global_batch": world if shard == "replicas" else 1, "seq_len": wl.N,
+            "parallelism": f"{shard} x{world}",
             "l2": "inputs larger than L2 (604 MB per tensor), no flush"}
 
 
@@ -241,7 +243,20 @@ def run_b200(args, rank, world, local):
     nB = math.ceil(N / 128)
 
     # ---- inputs (fresh per step, cycled from a pool), outputs, index buffers
-    pool = [inputs.workload_qkv(inputs_wl(wl, rank), s, device=dev) for s in range(POOL)]
+    H_total = wl.H
+    if args.shard == "heads":
+        # one problem split by heads: every rank draws the same inputs and keeps its head range
+        from block_sparse_attention_lvsa_b200 import heads
+        import dataclasses
+        h0, h1 = heads.head_range(wl.H, world, rank)
+        if h1 == h0:
+            raise SystemExit("--shard heads needs at least as many heads as ranks")
+        pool = [tuple(heads.local_heads(x, wl.H, world, rank) for x in inputs.workload_qkv(wl, s, device=dev))
+                for s in range(POOL)]
+        wl = dataclasses.replace(wl, H=h1 - h0)
+        H = wl.H
+    else:
+        pool = [inputs.workload_qkv(inputs_wl(wl, rank), s, device=dev) for s in range(POOL)]
     o = torch.empty_like(pool[0][0])
     lse = torch.empty((H, N), dtype=torch.float32, device=dev)
     frames = torch.empty((wl.T, wl.T), dtype=torch.int32, device=dev)
@@ -325,6 +340,7 @@ def run_b200(args, rank, world, local):
 
     # ---- balanced variant of the same shape (T_per = 21: |A(t)| = C = 21 for every t and s)
     balanced = run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws) if rank == 0 else None
+    gather = run_gather(o, lse, H_total, world) if args.shard == "heads" and world > 1 else None
 
     # ---- e2e: host buffers through the public API, copies inside the timed region
     e2e = run_e2e(bsa, wl, pool[0], stream, frames, counts, ix, o, lse, ws, max(2, min(args.steps, 10)),
@@ -338,8 +354,8 @@ def run_b200(args, rank, world, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_block(wl, world),
+        "scaling": "weak" if args.shard == "replicas" else "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_block(wl, world, args.shard, H_total),
         "ms_per_call": med_call,
         "tflops_kept_tiles": achieved,
         "tflops_exact_pairs": sum(flop_exact) / (sum(call_ms) / 1e3) / 1e12,
@@ -358,6 +374,8 @@ def run_b200(args, rank, world, local):
         "losa": losa,
         "balanced_tper21": balanced,
     }
+    if gather is not None:
+        line["gather_heads"] = gather
     if rank == 0 and not args.no_cpu_baseline:
         dt, fl, n, cores = oracle_sample(wl, 0, args.cpu_rows, head=0, qkv=None, seed=7)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -373,6 +391,25 @@ def run_b200(args, rank, world, local):
 # grows with the number of heads.  Must be re-measured (or set to None)
 # whenever the kernel changes.
 TRAFFIC_PER_LAUNCH = 2.607e9
+
+
+def run_gather(o, lse, H, world, reps=3):
+    """Time of assembling every rank's O and LSE shards on all ranks (one
+    all-gather per tensor; NCCL over NVLink), outside the attention path."""
+    from block_sparse_attention_lvsa_b200 import heads
+    ms = []
+    for i in range(reps + 1):
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        og, lg = heads.gather_heads(o, lse, H)
+        b.record()
+        torch.cuda.synchronize()
+        if i:
+            ms.append(max_over_ranks(a.elapsed_time(b), world))
+    nbytes = og.numel() * og.element_size() + lg.numel() * lg.element_size()
+    return {"ms": statistics.median(ms), "bytes_per_rank_out": nbytes,
+            "note": "not part of the timed steps; the path itself has no exchange"}
 
 
 def run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws, calls=6):
@@ -393,7 +430,7 @@ def run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws, calls=6):
         _, tcnt, _, _ = bsa.lvsa_workspace_views(ws, wl.N, wl.T)
         k = int(tcnt.sum().item())
         kept += k
-        flop += 4 * wl.d * wl.H * k * 128 * 128
+        flop += 4 * wl.d * pool[0][0].shape[1] * k * 128 * 128
         ms.append(a.elapsed_time(b))
     status = bsa.get_device_status()
     nB = math.ceil(wl.N / 128)
@@ -575,6 +612,8 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="profiling only: override the head count")
     ap.add_argument("--main-only", action="store_true", help="profiling only: timed LVSA steps, nothing else")
     ap.add_argument("--select-only", action="store_true", help="profiling only: the LoSA selection, small case")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: independent replicas (weak scaling) or one problem split by heads (strong)")
     args = ap.parse_args()
     if args.select_only:
         run_select_only()
