@@ -337,6 +337,8 @@ def run_b200(args, rank, world, local):
             dense_ms.append(a.elapsed_time(b))
     dense_ms = statistics.median(dense_ms)
     dense_flop = 4 * d * H * nB * nB * 128 * 128
+    sdpa = run_sdpa_context(pool[0], wl.scale, stream) if rank == 0 else None
+    index_us = graph_timed(lambda: bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, 1, frames, counts), 50) * 1e3
 
     # ---- balanced variant of the same shape (T_per = 21: |A(t)| = C = 21 for every t and s)
     balanced = run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws) if rank == 0 else None
@@ -373,6 +375,9 @@ def run_b200(args, rank, world, local):
         "clocks": clocks,
         "losa": losa,
         "balanced_tper21": balanced,
+        "lvsa_build_index": {"us": index_us, "bytes_out": (wl.T * wl.T + wl.T) * 4,
+                             "note": "a few KB written: latency-bound, GB/s not meaningful"},
+        "context_torch_sdpa_dense": sdpa,
     }
     if gather is not None:
         line["gather_heads"] = gather
@@ -380,7 +385,9 @@ def run_b200(args, rank, world, local):
         dt, fl, n, cores = oracle_sample(wl, 0, args.cpu_rows, head=0, qkv=None, seed=7)
         line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"{n} stratified query rows of head 0 at step 0 ({dt:.1f} s), fp64 numpy; "
-                                          "kept-tile-equivalent FLOPs"}
+                                          "kept-tile-equivalent FLOPs",
+                                "rows_per_s": n / dt,
+                                "extrapolated_full_call_s": dt * wl.N * H_total / n}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -410,6 +417,28 @@ def run_gather(o, lse, H, world, reps=3):
     nbytes = og.numel() * og.element_size() + lg.numel() * lg.element_size()
     return {"ms": statistics.median(ms), "bytes_per_rank_out": nbytes,
             "note": "not part of the timed steps; the path itself has no exchange"}
+
+
+def run_sdpa_context(qkv, scale, stream, reps=2):
+    """Context only (a library kernel, not part of this path): torch's
+    scaled_dot_product_attention, dense, on the same q, k, v."""
+    import torch.nn.functional as F
+    q, k, v = (x.transpose(0, 1).unsqueeze(0) for x in qkv)       # [1, H, N, d] views
+    try:
+        ms = []
+        for i in range(reps + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            out = F.scaled_dot_product_attention(q, k, v, scale=scale)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i:
+                ms.append(a.elapsed_time(b))
+        del out
+        N, H, d = qkv[0].shape
+        return {"ms": statistics.median(ms), "tflops": 4 * d * H * N * N / (statistics.median(ms) / 1e3) / 1e12}
+    except Exception as e:                                        # noqa: BLE001 - context only
+        return {"unavailable": str(e).splitlines()[0][:200]}
 
 
 def run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws, calls=6):
@@ -604,7 +633,7 @@ def run_select_only():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--cpu-rows", type=int, default=16384)

@@ -232,8 +232,39 @@ __device__ __forceinline__ float exp2_poly3(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
-// columns of the 128 computed with exp2_poly3 in unmasked tiles (0: all on MUFU)
+// Of every 8 columns of an unmasked tile, kPolyCols / 16 take exp2_poly3 on
+// the FMA pipe and the rest ex2 on MUFU (masked tiles stay on MUFU: the
+// polynomial does not give exactly 0 for a masked score).  Off: FMA-dense
+// code in a softmax warp that shares a sub-partition with the MMA-issuing
+// thread slows the issue of every tcgen05.mma (measured: 64 -> ~120 cycles
+// per 128x128x16 MMA next to a warp issuing an FFMA per cycle), and every
+// sub-partition holds softmax warps; 16, 32 and 48 columns measured 10-20%
+// slower overall.
 constexpr int kPolyCols = 0;
+
+// exp2(s * sl2 - m) for one 128-score row; P (bf16 pairs) packed in place
+// into sr[0..63] (pair j overwrites sr[j] only after elements 2j, 2j+1 >= j
+// are read).  Returns the row sum of the float32 values.
+template <int NPOLY>
+__device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use) {
+  float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 128; c += 4) {
+    float e[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float xx = fmaf(s[c + u], sl2, -m_use);
+      e[u] = (((c + u) & 7) * 16 < NPOLY) ? exp2_poly3(xx) : ex2_approx(xx);
+    }
+    rs0 += e[0];
+    rs1 += e[1];
+    rs2 += e[2];
+    rs3 += e[3];
+    sr[c / 2] = pack_bf16x2(e[0], e[1]);
+    sr[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
+  }
+  return (rs0 + rs1) + (rs2 + rs3);
+}
 
 template <int D, bool MASS>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -533,27 +564,10 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
           }
         }
-        // p = exp2(s * scale * log2e - m); P (bf16 pairs) packed in place into sr[0..63]
-        // (pair j overwrites sr[j] only after elements 2j, 2j+1 >= j are read)
-        float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-        const bool poly = !part;
-#pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          float e[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float xx = fmaf(s[c + u], p.sl2, -m_use);
-            e[u] = (kPolyCols > 0 && poly && (c + u) < kPolyCols) ? exp2_poly3(xx) : ex2_approx(xx);
-          }
-          rs0 += e[0];
-          rs1 += e[1];
-          rs2 += e[2];
-          rs3 += e[3];
-          sr[c / 2] = pack_bf16x2(e[0], e[1]);
-          sr[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
-        }
+        // p = exp2(s * scale * log2e - m), P packed in place (the tile's flag is
+        // the same for the whole group: no divergence)
+        const float rsum = part ? row_exp_pack<0>(s, sr, p.sl2, m_use) : row_exp_pack<kPolyCols>(s, sr, p.sl2, m_use);
         tmem_st_x64(tS, sr);
-        const float rsum = (rs0 + rs1) + (rs2 + rs3);
         if constexpr (MASS) {
           // this tile's share of the row's mass, log2, before normalisation
           if (q < p.N)
