@@ -136,6 +136,35 @@ def block_mass(q: np.ndarray, k: np.ndarray, scale: float, block: int,
     return out
 
 
+def block_mass_restricted(q: np.ndarray, k: np.ndarray, scale: float, block: int,
+                          heads: Iterable[int], qblocks: Iterable[int],
+                          allowed: Callable[[int, int], np.ndarray]) -> Dict[Tuple[int, int], np.ndarray]:
+    """mass[h, qb, :] of attention restricted to allowed key sets.
+
+    The LoSA measuring step ([LoSA] "Balancing efficiency and quality") run
+    on attention that is already restricted, e.g. to LVSA's frames A(t)
+    ([LVSA] sec. 2): p_h(q, k) is the softmax of q over allowed(h, q) only
+    (zero elsewhere) and the mass of (qb, kb) sums it over the rectangle.
+    Rows with no allowed key contribute nothing.
+    """
+    N = q.shape[0]
+    nB = -(-N // block)
+    out = {}
+    for h in heads:
+        for qb in qblocks:
+            mass = np.zeros(nB)
+            for r in range(qb * block, min((qb + 1) * block, N)):
+                keys = np.asarray(allowed(h, r), dtype=np.int64)
+                if keys.size == 0:
+                    continue
+                s = (k[keys, h, :] @ q[r, h, :]) * scale
+                e = np.exp(s - s.max())
+                e /= e.sum()
+                np.add.at(mass, keys // block, e)
+            out[(h, qb)] = mass
+    return out
+
+
 def block_mass_from_probabilities(p: np.ndarray, block: int) -> np.ndarray:
     """mass [nB, nB] from an explicit [N, N] probability matrix (brute force, small N)."""
     N = p.shape[0]

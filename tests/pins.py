@@ -303,6 +303,50 @@ def check_block_mass(attention):
             assert abs(got[(0, qb)][kb] - sizes[qb] * sizes[kb] / N) < 1e-12
 
 
+def check_block_mass_restricted(attention, lvsa):
+    """Block mass of frame-restricted attention: the library softmax over the
+    masked score matrix, summed over rectangles in the test; rows sum to 1
+    (rows with an allowed key); nothing outside allowed blocks; dense sets
+    give the dense mass; q = 0 gives the closed form."""
+    rng = np.random.default_rng(11)
+    T, P, H, d, blk = 6, 70, 2, 16, 128                 # N = 420: 4 blocks, ragged last (36 rows)
+    N = T * P
+    q, k = rng.standard_normal((N, H, d)), rng.standard_normal((N, H, d))
+    scale = 0.35
+    nB = -(-N // blk)
+    edges = np.arange(0, N, blk)
+    for dense in (False, True):
+        A = [list(range(T))] * T if dense else random_allowed(T, rng, 0.3)
+        mask = lvsa.dense_token_mask(A, P, N)
+        allowed = lambda h, r: lvsa.allowed_keys_for_row(r, A, P, N)     # noqa: E731
+        got = attention.block_mass_restricted(q, k, scale, blk, range(H), range(nB), allowed)
+        for h in range(H):
+            S = torch.from_numpy(q[:, h] @ k[:, h].T * scale).masked_fill(~torch.from_numpy(mask), float("-inf"))
+            p = torch.softmax(S, dim=-1).numpy()                         # library softmax
+            p = np.nan_to_num(p)                                         # rows without keys: none here
+            rect = np.add.reduceat(np.add.reduceat(p, edges, axis=0), edges, axis=1)
+            for qb in range(nB):
+                assert np.allclose(got[(h, qb)], rect[qb], atol=1e-12), (dense, h, qb)
+                rows = min((qb + 1) * blk, N) - qb * blk
+                assert abs(got[(h, qb)].sum() - rows) < 1e-9
+                blk_allowed = mask[qb * blk:(qb + 1) * blk].reshape(-1, N).any(axis=0)
+                for kb in range(nB):
+                    if not blk_allowed[kb * blk:(kb + 1) * blk].any():
+                        assert got[(h, qb)][kb] == 0.0
+            if dense:
+                ref = attention.block_mass(q, k, scale, blk, [h], range(nB))
+                for qb in range(nB):
+                    assert np.allclose(got[(h, qb)], ref[(h, qb)], atol=1e-12)
+        # q == 0: uniform over each row's allowed keys
+        got = attention.block_mass_restricted(np.zeros_like(q), k, scale, blk, [0], range(nB), allowed)
+        for qb in range(nB):
+            want = np.zeros(nB)
+            for r in range(qb * blk, min((qb + 1) * blk, N)):
+                keys = np.flatnonzero(mask[r])
+                np.add.at(want, keys // blk, 1.0 / keys.size)
+            assert np.allclose(got[(0, qb)], want, atol=1e-12)
+
+
 # ----------------------------------------------------------------- LoSA ---
 def read_losa_golden():
     cases = []

@@ -17,3 +17,7 @@ def test_triple_loop():
 
 def test_block_mass():
     pins.check_block_mass(attention)
+
+
+def test_block_mass_restricted():
+    pins.check_block_mass_restricted(attention, lvsa)

@@ -111,6 +111,28 @@ def test_lvsa_window_mistakes_caught(kind):
     assert fails(pins.check_lvsa_window_bruteforce, m)
 
 
+def test_restricted_mass_normaliser_caught():
+    m = clone(attention)
+
+    def restricted(q, k, scale, block, heads, qblocks, allowed):
+        N = q.shape[0]
+        nB = -(-N // block)
+        out = {}
+        for h in heads:
+            for qb in qblocks:
+                mass = np.zeros(nB)
+                for r in range(qb * block, min((qb + 1) * block, N)):
+                    keys = np.asarray(allowed(h, r), dtype=np.int64)
+                    s_all = (k[:, h, :] @ q[r, h, :]) * scale
+                    e = np.exp(s_all - s_all.max())
+                    e /= e.sum()                          # normalised over every key: wrong
+                    np.add.at(mass, keys // block, e[keys])
+                out[(h, qb)] = mass
+        return out
+    m.block_mass_restricted = restricted
+    assert fails(pins.check_block_mass_restricted, m, lvsa)
+
+
 def test_tiles_partial_flag_caught():
     m = clone(tiles)
 
