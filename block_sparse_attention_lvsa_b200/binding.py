@@ -30,10 +30,12 @@ BSA_ERR_WORKSPACE = -7
 
 BSA_INDEX_LVSA_FRAMES = 1
 BSA_INDEX_BLOCKS = 2
+BSA_INDEX_LVSA_BLOCKS = 3
 BSA_OP_BLOCKSPARSE_FWD = 1
 BSA_OP_DENSE_BLOCKMASS = 2
+BSA_OP_BLOCKMASS = 3
 
-EXPORTED = ("lvsa_build_index", "lvsa_build_index_window", "attn_dense_blockmass", "losa_select", "blocksparse_attn_fwd",
+EXPORTED = ("lvsa_build_index", "lvsa_build_index_window", "attn_dense_blockmass", "attn_blockmass", "losa_select", "blocksparse_attn_fwd",
             "bsa_workspace_bytes", "bsa_get_device_status", "bsa_status_string",
             "bsa_debug_expired_wait", "bsa_version", "blocksparse_attn_fwd_noalloc")
 
@@ -71,6 +73,7 @@ def _load():
         "lvsa_build_index": (I, [I, I, I, I, I, P, P, P]),
         "lvsa_build_index_window": (I, [I, I, I, I, P, P, P]),
         "attn_dense_blockmass": (I, [P, P, P, I, I, I, I, F, P, P, P, P, SZ, P]),
+        "attn_blockmass": (I, [P, P, P, I, I, I, F, ctypes.POINTER(bsa_index), P, P, P, P, SZ, P]),
         "losa_select": (I, [P, I, I, I, D, P, P, P]),
         "blocksparse_attn_fwd": (I, [P, P, P, I, I, I, F, ctypes.POINTER(bsa_index), P, P, P, SZ, P]),
         "bsa_workspace_bytes": (SZ, [I, I, I, I, ctypes.POINTER(bsa_index)]),
@@ -176,6 +179,17 @@ def block_index(idx: torch.Tensor, cnt: torch.Tensor, block: int = 128) -> bsa_i
     return ix
 
 
+def lvsa_block_index(T: int, frames: torch.Tensor, counts: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor,
+                     block: int = 128) -> bsa_index:
+    """Intersection index: LVSA frame sets (frames, counts) within per-head key-block lists (idx, cnt)."""
+    ix = block_index(idx, cnt, block)
+    ix.kind = BSA_INDEX_LVSA_BLOCKS
+    ix.T = T
+    ix.frames = frames.data_ptr()
+    ix.counts = counts.data_ptr()
+    return ix
+
+
 def workspace_bytes(op: int, N: int, H: int, d: int, index: Optional[bsa_index] = None) -> int:
     n = _lib.bsa_workspace_bytes(op, N, H, d, ctypes.byref(index) if index is not None else None)
     if n == ctypes.c_size_t(-1).value:
@@ -248,6 +262,30 @@ def attn_dense_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bloc
                                    _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel(),
                                    _stream(stream))
     _check("attn_dense_blockmass", rc)
+    return o, lse, mass
+
+
+def attn_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, index: bsa_index,
+                   scale: Optional[float] = None, o=None, lse=None, mass=None,
+                   workspace: Optional[torch.Tensor] = None, stream=None):
+    """Attention restricted to ``index`` plus its LoSA block mass; returns (o, lse, mass [H, nB, nB] f32)."""
+    _check_qkv(q, k, v)
+    N, H, d = q.shape
+    nB = math.ceil(N / 128)
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, N), dtype=torch.float32, device=q.device)
+    if mass is None:
+        mass = torch.empty((H, nB, nB), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(BSA_OP_BLOCKMASS, N, H, d, index), dtype=torch.uint8,
+                                device=q.device)
+    rc = _lib.attn_blockmass(_ptr(q), _ptr(k), _ptr(v), N, H, d, float(scale), ctypes.byref(index),
+                             _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("attn_blockmass", rc)
     return o, lse, mass
 
 

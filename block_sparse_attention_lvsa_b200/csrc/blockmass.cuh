@@ -39,7 +39,9 @@ blockmass_reduce_kernel(const float* __restrict__ lpart, const float* __restrict
     if (q < N) {
       const float v = lp[q];
       const float l2 = ls[q] * 1.4426950408889634f;
-      if (v != -INFINITY && l2 != -INFINITY) acc += ex2_approx(v - l2);
+      // -inf: no allowed key of the tile in this row; NaN: a tile the index
+      // never reached (the workspace was set to NaN first); lse -inf: an empty row
+      if (v > -INFINITY && l2 > -INFINITY) acc += ex2_approx(v - l2);
     }
   }
 #pragma unroll

@@ -118,6 +118,30 @@ AttnParams base_params(int N, int H, float scale, void* o, float* lse) {
 // sums [nB key tiles][N rows] float32.
 size_t dense_mass_head_bytes(int N) { return static_cast<size_t>(n_tiles(N)) * static_cast<size_t>(N) * 4; }
 
+// Forward in mass mode over head passes of `hc` heads, each followed by the
+// block-mass reduction.  With `unvisited`, the log partial sums are first
+// set to NaN (all bytes 0xFF): entries of tiles the index never reaches keep
+// it and the reduction counts them as no mass.
+int blockmass_passes(const void* q, const void* k, const void* v, int N, int H, int d, AttnParams p, float* lpart,
+                     int hc, bool unvisited, const float* lse, float* mass, cudaStream_t st) {
+  const int nB = n_tiles(N);
+  const size_t per_head = dense_mass_head_bytes(N);
+  for (int h0 = 0; h0 < H; h0 += hc) {
+    const int hn = std::min(hc, H - h0);
+    if (unvisited && cudaMemsetAsync(lpart, 0xFF, per_head * hn, st) != cudaSuccess) return BSA_ERR_CUDA;
+    p.lpart = lpart;
+    p.h_off = h0;
+    int rc = launch_attn_any(d, true, q, k, v, N, H, hn, p, st);
+    if (rc != BSA_OK) return rc;
+    const long long warps = static_cast<long long>(hn) * nB * nB;
+    const long long blocks = (warps + kMassThreads / 32 - 1) / (kMassThreads / 32);
+    if (blocks > 0x7FFFFFFFLL) return BSA_ERR_UNSUPPORTED;
+    blockmass_reduce_kernel<<<static_cast<unsigned>(blocks), kMassThreads, 0, st>>>(lpart, lse, mass, N, nB, h0, hn);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
+}
+
 // Workspace layout for LVSA frame indexes.
 struct LvsaWs {
   size_t fbits, cnt, idx, flag, total;
@@ -132,6 +156,77 @@ LvsaWs lvsa_ws_layout(int N, int T) {
   w.flag = round_up(w.idx + nB * nB * 4, 256);
   w.total = round_up(w.flag + nB * nB, 256);
   return w;
+}
+
+// Workspace bytes an index needs (LVSA tile lists; for the intersection also
+// its per-entry flags [H][nB][nB]); (size_t)-1 for an invalid index.
+size_t index_ws_bytes(const bsa_index* index, int N, int H) {
+  if (!index) return static_cast<size_t>(-1);
+  if (index->kind == BSA_INDEX_BLOCKS) return 0;
+  if (index->kind != BSA_INDEX_LVSA_FRAMES && index->kind != BSA_INDEX_LVSA_BLOCKS) return static_cast<size_t>(-1);
+  if (index->T < 1 || index->T > kMaxFrames || N % index->T) return static_cast<size_t>(-1);
+  const size_t nB = static_cast<size_t>(n_tiles(N));
+  size_t t = lvsa_ws_layout(N, index->T).total;
+  if (index->kind == BSA_INDEX_LVSA_BLOCKS) t += round_up(static_cast<size_t>(H) * nB * nB, 256);
+  return t;
+}
+
+// Validates `index`, enqueues its expansion (LVSA frame sets -> tile lists,
+// flags of the intersection) and fills the list fields of `p`; *used = the
+// workspace bytes taken from its start.
+int setup_index(const bsa_index* index, int N, int H, void* workspace, size_t ws_bytes, AttnParams& p,
+                size_t* used, cudaStream_t st) {
+  const int nB = p.nB;
+  *used = 0;
+  const bool lvsa = index->kind == BSA_INDEX_LVSA_FRAMES || index->kind == BSA_INDEX_LVSA_BLOCKS;
+  const bool blocks = index->kind == BSA_INDEX_BLOCKS || index->kind == BSA_INDEX_LVSA_BLOCKS;
+  if (!lvsa && !blocks) return BSA_ERR_ARG;
+  if (blocks) {
+    if (index->block != 128) return BSA_ERR_UNSUPPORTED;
+    if (index->H != H || index->nQB != nB || index->nKB != nB) return BSA_ERR_SHAPE;
+    if (!index->idx || !index->cnt) return BSA_ERR_ARG;
+    p.list = index->idx;
+    p.count = index->cnt;
+    p.flags = nullptr;
+    p.lhs = static_cast<long long>(index->nQB) * index->nKB;
+    p.lrs = index->nKB;
+    p.chs = index->nQB;
+  }
+  if (lvsa) {
+    const int T = index->T;
+    if (T < 1 || T > kMaxFrames) return BSA_ERR_ARG;
+    if (N % T) return BSA_ERR_SHAPE;
+    if (!index->frames || !index->counts) return BSA_ERR_ARG;
+    const LvsaWs w = lvsa_ws_layout(N, T);
+    const size_t need = index_ws_bytes(index, N, H);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return BSA_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint32_t* fbits = reinterpret_cast<uint32_t*>(ws + w.fbits);
+    int32_t* tcnt = reinterpret_cast<int32_t*>(ws + w.cnt);
+    int32_t* tidx = reinterpret_cast<int32_t*>(ws + w.idx);
+    uint8_t* tflag = ws + w.flag;
+    lvsa_frame_bits_kernel<<<(T + 127) / 128, 128, 0, st>>>(T, index->frames, index->counts, fbits);
+    lvsa_tiles_kernel<<<(nB + 3) / 4, 128, 0, st>>>(N, T, N / T, nB, fbits, tcnt, tidx, tflag);
+    p.fbits = fbits;
+    p.TW = (T + 31) / 32;
+    p.P = N / T;
+    if (blocks) {
+      uint8_t* cflag = ws + w.total;
+      compose_flags_kernel<<<static_cast<unsigned>(H) * nB, 256, 0, st>>>(nB, index->idx, index->cnt, tcnt, tidx,
+                                                                        tflag, cflag);
+      p.flags = cflag;
+    } else {
+      p.list = tidx;
+      p.count = tcnt;
+      p.flags = tflag;
+      p.lhs = 0;
+      p.lrs = nB;
+      p.chs = 0;
+    }
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    *used = need;
+  }
+  return BSA_OK;
 }
 
 }  // namespace
@@ -182,17 +277,14 @@ int lvsa_build_index_window(int T, int T_per, int W, int step, int32_t* frames, 
 
 size_t bsa_workspace_bytes(int op, int N, int H, int d, const bsa_index* index) {
   if (N < 1 || H < 1 || (d != 64 && d != 128)) return static_cast<size_t>(-1);
-  if (op == BSA_OP_DENSE_BLOCKMASS) {
-    // every head in one pass, up to 4 GiB; any multiple of one head's share works
-    const size_t per_head = dense_mass_head_bytes(N);
-    const size_t heads = std::max<size_t>(1, std::min<size_t>(static_cast<size_t>(H), (size_t(4) << 30) / per_head));
-    return per_head * heads;
-  }
-  if (op != BSA_OP_BLOCKSPARSE_FWD || !index) return static_cast<size_t>(-1);
-  if (index->kind == BSA_INDEX_BLOCKS) return 0;
-  if (index->kind != BSA_INDEX_LVSA_FRAMES || index->T < 1 || index->T > kMaxFrames || N % index->T)
-    return static_cast<size_t>(-1);
-  return lvsa_ws_layout(N, index->T).total;
+  const size_t per_head = dense_mass_head_bytes(N);
+  // head shares of log partial sums: every head in one pass, up to 4 GiB
+  const size_t heads = std::max<size_t>(1, std::min<size_t>(static_cast<size_t>(H), (size_t(4) << 30) / per_head));
+  if (op == BSA_OP_DENSE_BLOCKMASS) return per_head * heads;
+  if (op != BSA_OP_BLOCKSPARSE_FWD && op != BSA_OP_BLOCKMASS) return static_cast<size_t>(-1);
+  const size_t ix = index_ws_bytes(index, N, H);
+  if (ix == static_cast<size_t>(-1)) return ix;
+  return op == BSA_OP_BLOCKSPARSE_FWD ? ix : round_up(ix, 256) + per_head * heads;
 }
 
 int blocksparse_attn_fwd(const void* q, const void* k, const void* v, int N, int H, int d, float scale,
@@ -203,45 +295,29 @@ int blocksparse_attn_fwd(const void* q, const void* k, const void* v, int N, int
   if (!index || !std::isfinite(scale)) return BSA_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   AttnParams p = base_params(N, H, scale, o, lse);
-  const int nB = p.nB;
-  if (index->kind == BSA_INDEX_LVSA_FRAMES) {
-    const int T = index->T;
-    if (T < 1 || T > kMaxFrames) return BSA_ERR_ARG;
-    if (N % T) return BSA_ERR_SHAPE;
-    if (!index->frames || !index->counts) return BSA_ERR_ARG;
-    const LvsaWs w = lvsa_ws_layout(N, T);
-    if (!workspace || ws_bytes < w.total || !aligned(workspace, 256)) return BSA_ERR_WORKSPACE;
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    uint32_t* fbits = reinterpret_cast<uint32_t*>(ws + w.fbits);
-    int32_t* tcnt = reinterpret_cast<int32_t*>(ws + w.cnt);
-    int32_t* tidx = reinterpret_cast<int32_t*>(ws + w.idx);
-    uint8_t* tflag = ws + w.flag;
-    lvsa_frame_bits_kernel<<<(T + 127) / 128, 128, 0, st>>>(T, index->frames, index->counts, fbits);
-    lvsa_tiles_kernel<<<(nB + 3) / 4, 128, 0, st>>>(N, T, N / T, nB, fbits, tcnt, tidx, tflag);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-    p.list = tidx;
-    p.count = tcnt;
-    p.flags = tflag;
-    p.lhs = 0;
-    p.lrs = nB;
-    p.chs = 0;
-    p.fbits = fbits;
-    p.TW = (T + 31) / 32;
-    p.P = N / T;
-  } else if (index->kind == BSA_INDEX_BLOCKS) {
-    if (index->block != 128) return BSA_ERR_UNSUPPORTED;
-    if (index->H != H || index->nQB != nB || index->nKB != nB) return BSA_ERR_SHAPE;
-    if (!index->idx || !index->cnt) return BSA_ERR_ARG;
-    p.list = index->idx;
-    p.count = index->cnt;
-    p.flags = nullptr;
-    p.lhs = static_cast<long long>(index->nQB) * index->nKB;
-    p.lrs = index->nKB;
-    p.chs = index->nQB;
-  } else {
-    return BSA_ERR_ARG;
-  }
+  size_t used = 0;
+  rc = setup_index(index, N, H, workspace, ws_bytes, p, &used, st);
+  if (rc != BSA_OK) return rc;
   return launch_attn_any(d, false, q, k, v, N, H, H, p, st);
+}
+
+int attn_blockmass(const void* q, const void* k, const void* v, int N, int H, int d, float scale,
+                   const bsa_index* index, void* o, float* lse, float* mass, void* workspace, size_t ws_bytes,
+                   void* stream) {
+  int rc = check_qkv(q, k, v, N, H, d, o, lse);
+  if (rc != BSA_OK) return rc;
+  if (!index || !mass || !aligned(mass, 4) || !std::isfinite(scale)) return BSA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  AttnParams p = base_params(N, H, scale, o, lse);
+  size_t used = 0;
+  rc = setup_index(index, N, H, workspace, ws_bytes, p, &used, st);
+  if (rc != BSA_OK) return rc;
+  const size_t off = round_up(used, 256);
+  const size_t per_head = dense_mass_head_bytes(N);
+  if (!workspace || ws_bytes < off || ws_bytes - off < per_head) return BSA_ERR_WORKSPACE;
+  float* lpart = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + off);
+  const int hc = static_cast<int>(std::min<size_t>(static_cast<size_t>(H), (ws_bytes - off) / per_head));
+  return blockmass_passes(q, k, v, N, H, d, p, lpart, hc, /*unvisited=*/true, lse, mass, st);
 }
 
 int attn_dense_blockmass(const void* q, const void* k, const void* v, int N, int H, int d, int block, float scale,
@@ -252,27 +328,12 @@ int attn_dense_blockmass(const void* q, const void* k, const void* v, int N, int
   if (block != 128) return BSA_ERR_UNSUPPORTED;
   const size_t per_head = dense_mass_head_bytes(N);
   if (!workspace || !aligned(workspace, 256) || ws_bytes < per_head) return BSA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int nB = n_tiles(N);
-  // as many heads per pass as the workspace holds: the forward writes their
-  // log partial sums, the reduction turns them into block mass
+  AttnParams p = base_params(N, H, scale, o, lse);
+  p.dense = 1;
   const int hc = static_cast<int>(std::min<size_t>(static_cast<size_t>(H), ws_bytes / per_head));
-  for (int h0 = 0; h0 < H; h0 += hc) {
-    const int hn = std::min(hc, H - h0);
-    AttnParams p = base_params(N, H, scale, o, lse);
-    p.dense = 1;
-    p.lpart = static_cast<float*>(workspace);
-    p.h_off = h0;
-    rc = launch_attn_any(d, true, q, k, v, N, H, hn, p, st);
-    if (rc != BSA_OK) return rc;
-    const long long warps = static_cast<long long>(hn) * nB * nB;
-    const long long blocks = (warps + kMassThreads / 32 - 1) / (kMassThreads / 32);
-    if (blocks > 0x7FFFFFFFLL) return BSA_ERR_UNSUPPORTED;
-    blockmass_reduce_kernel<<<static_cast<unsigned>(blocks), kMassThreads, 0, st>>>(
-        static_cast<const float*>(workspace), lse, mass, N, nB, h0, hn);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-  }
-  return BSA_OK;
+  // every (row, key tile) is visited: no need to mark the workspace first
+  return blockmass_passes(q, k, v, N, H, d, p, static_cast<float*>(workspace), hc, false, lse, mass,
+                          static_cast<cudaStream_t>(stream));
 }
 
 int losa_select(const float* mass, int H, int nQB, int nKB, double tau, int32_t* idx, int32_t* cnt, void* stream) {

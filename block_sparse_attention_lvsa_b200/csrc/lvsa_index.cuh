@@ -139,4 +139,35 @@ __global__ void lvsa_tiles_kernel(int N, int T, int P, int nB, const uint32_t* _
   if (lane == 0) tile_cnt[qt] = total;
 }
 
+// Per-entry partial flags of a block index intersected with LVSA frames.
+// Entry (h, qb, j < cnt[h][qb]) keeps key tile kt = idx[h][qb][j].  Pairs of
+// that tile stay subject to the LVSA element rule, so the tile is whole only
+// if LVSA keeps it whole for query tile qb: its flag is the one in qb's LVSA
+// tile list (found by binary search: the lists are ascending).  A tile the
+// LVSA list does not hold is marked partial; its element mask then admits
+// none of its pairs.  One block per (h, qb) row.
+__global__ void compose_flags_kernel(int nB, const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
+                                     const int32_t* __restrict__ tile_cnt, const int32_t* __restrict__ tile_idx,
+                                     const uint8_t* __restrict__ tile_flag, uint8_t* __restrict__ flags) {
+  const size_t row = blockIdx.x;                        // h * nB + qb
+  const int qb = static_cast<int>(row % nB);
+  const int c = min(max(cnt[row], 0), nB);
+  const int n = min(max(tile_cnt[qb], 0), nB);
+  const int32_t* lv = tile_idx + static_cast<size_t>(qb) * nB;
+  for (int j = threadIdx.x; j < nB; j += blockDim.x) {
+    uint8_t f = 0;
+    if (j < c) {
+      f = 1;
+      const int kt = idx[row * nB + j];
+      int lo = 0, hi = n;                               // first position with lv[pos] >= kt
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (lv[mid] < kt) lo = mid + 1; else hi = mid;
+      }
+      if (lo < n && lv[lo] == kt) f = tile_flag[static_cast<size_t>(qb) * nB + lo];
+    }
+    flags[row * nB + j] = f;
+  }
+}
+
 }  // namespace bsa

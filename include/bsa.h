@@ -63,7 +63,8 @@ typedef enum bsa_status {
 /* Index kinds accepted by blocksparse_attn_fwd. */
 enum {
   BSA_INDEX_LVSA_FRAMES = 1,  /* frame lists from lvsa_build_index          */
-  BSA_INDEX_BLOCKS = 2        /* key-block lists from losa_select           */
+  BSA_INDEX_BLOCKS = 2,       /* key-block lists from losa_select           */
+  BSA_INDEX_LVSA_BLOCKS = 3   /* both: LVSA frames within selected blocks   */
 };
 
 /*
@@ -84,6 +85,11 @@ enum {
  *   (h, q / 128).  Entries outside [0, nKB) are skipped and reported as
  *   BSA_ERR_INDEX_RANGE through the device status word; a count outside
  *   [0, nKB] is clamped and reported the same way.
+ * kind == BSA_INDEX_LVSA_BLOCKS (all fields of kinds 1 and 2): the
+ *   intersection - query token q of head h may attend key token k iff
+ *   frame(k) is in A(frame(q)) and k / 128 is listed in row (h, q / 128).
+ *   This runs LoSA's per-head block selection inside LVSA's frame sets; the
+ *   pages never combine the two methods, so it is offered as a variant.
  */
 typedef struct bsa_index {
   int kind;
@@ -170,6 +176,33 @@ int attn_dense_blockmass(const void* q, const void* k, const void* v,
                          int N, int H, int d, int block, float scale,
                          void* o, float* lse, float* mass,
                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * attn_blockmass - attention restricted to an index that also emits the
+ * LoSA block mass of that restricted attention.
+ *
+ * Source: [LoSA] section "Balancing efficiency and quality" (the measuring
+ * step records the attention mass between blocks), applied to attention
+ * already restricted by `index` (e.g. LVSA frames, [LVSA] section 2), so
+ * that a LoSA selection can be made inside the LVSA sets.  o and lse are
+ * those of blocksparse_attn_fwd with the same index; mass[h,qb,kb] sums the
+ * restricted float32 probabilities over the (qb, kb) rectangle (0 for
+ * blocks the index does not reach).  attn_dense_blockmass is the case of
+ * the full index.
+ *
+ * index: any kind accepted by blocksparse_attn_fwd.  workspace: device,
+ * 256-byte aligned, at least bsa_workspace_bytes(BSA_OP_BLOCKSPARSE_FWD,
+ * ...) rounded up to 256 plus one head's share of log partial sums
+ * (ceil(N/128) * N * 4 bytes); heads are processed in passes of as many
+ * shares as fit.  bsa_workspace_bytes(BSA_OP_BLOCKMASS, ...) gives all heads
+ * in one pass up to 4 GiB.  Other arguments as for attn_dense_blockmass.
+ * Returns BSA_OK or a negative bsa_status (BSA_ERR_WORKSPACE when the
+ * workspace is too small or misaligned).
+ */
+int attn_blockmass(const void* q, const void* k, const void* v,
+                   int N, int H, int d, float scale, const bsa_index* index,
+                   void* o, float* lse, float* mass,
+                   void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * losa_select - per (head, query block) minimal key-block set holding
@@ -263,7 +296,8 @@ int blocksparse_attn_fwd_noalloc(const void* q, const void* k, const void* v,
 /* Operation codes for bsa_workspace_bytes. */
 enum {
   BSA_OP_BLOCKSPARSE_FWD = 1,
-  BSA_OP_DENSE_BLOCKMASS = 2
+  BSA_OP_DENSE_BLOCKMASS = 2,
+  BSA_OP_BLOCKMASS = 3
 };
 
 /*

@@ -65,6 +65,18 @@ def test_workspace_bytes(bsa):
     ix.T = 7
     with pytest.raises(bsa.BsaError):      # T does not divide N
         bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 100, 1, 128, ix)
+    # intersection: the LVSA lists plus one flag byte per (head, query block, key block)
+    ix.kind, ix.T = bsa.BSA_INDEX_LVSA_FRAMES, 126
+    lv = bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 196560, 12, 128, ix)
+    ix.kind = bsa.BSA_INDEX_LVSA_BLOCKS
+    both = bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, 196560, 12, 128, ix)
+    assert both == lv + 12 * 1536 * 1536
+    # restricted mass: index part (256-aligned) + one share of log partial sums per head, all 12 here
+    share = 1536 * 196560 * 4
+    assert bsa.workspace_bytes(bsa.BSA_OP_BLOCKMASS, 196560, 12, 128, ix) == both + 1 * share or \
+        bsa.workspace_bytes(bsa.BSA_OP_BLOCKMASS, 196560, 12, 128, ix) == both + (4 << 30) // share * share
+    ix.kind = bsa.BSA_INDEX_BLOCKS
+    assert bsa.workspace_bytes(bsa.BSA_OP_BLOCKMASS, 32760, 40, 128, ix) == 40 * 256 * 32760 * 4
 
 
 def test_host_validation_rejects_before_launch(bsa):
@@ -112,6 +124,17 @@ def test_host_validation_rejects_before_launch(bsa):
     # the one-pass mass needs at least one head's share of workspace: 4 key tiles x 512 rows x 4 bytes
     assert g(fake, fake, fake, 512, 2, 64, 128, 0.1, fake, fake, fake, nul, 0, nul) == bsa.BSA_ERR_WORKSPACE
     assert g(fake, fake, fake, 512, 2, 64, 128, 0.1, fake, fake, fake, fake, 4 * 512 * 4 - 1, nul) == bsa.BSA_ERR_WORKSPACE
+    m = L.attn_blockmass
+    assert m(fake, fake, fake, 512, 2, 64, 0.1, None, fake, fake, fake, fake, 1 << 20, nul) == bsa.BSA_ERR_ARG
+    bix = bsa.bsa_index()
+    bix.kind = bsa.BSA_INDEX_LVSA_BLOCKS
+    bix.T, bix.frames, bix.counts = 8, 0x10000, 0x10000
+    bix.block, bix.H, bix.nQB, bix.nKB, bix.idx, bix.cnt = 128, 3, 4, 4, 0x10000, 0x10000
+    assert m(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(bix), fake, fake, fake, fake, 1 << 20, nul) == \
+        bsa.BSA_ERR_SHAPE                                   # H of the block lists != H
+    bix.H = 2
+    assert m(fake, fake, fake, 512, 2, 64, 0.1, ctypes.byref(bix), fake, fake, fake, fake, 100, nul) == \
+        bsa.BSA_ERR_WORKSPACE                               # too small for the lists, before any launch
     s = L.losa_select
     assert s(fake, 2, 4, 4, 0.0, fake, fake, nul) == bsa.BSA_ERR_ARG
     assert s(fake, 2, 4, 4, 1.5, fake, fake, nul) == bsa.BSA_ERR_ARG
