@@ -349,8 +349,9 @@ def run_b200(args, rank, world, local):
                   kept_tiles, world)
     del pool
 
-    # ---- LoSA path on the 14B-shaped workload (secondary measurements)
+    # ---- LoSA path on the 14B-shaped workload, and LoSA inside LVSA at 720p (secondary)
     losa = run_losa(bsa, rank, stream, peaks) if rank == 0 else None
+    lvsa_losa = run_lvsa_losa(bsa, stream) if rank == 0 else None
 
     med_call = statistics.median(call_ms)
     line = {
@@ -375,6 +376,7 @@ def run_b200(args, rank, world, local):
         "clocks": clocks,
         "losa": losa,
         "balanced_tper21": balanced,
+        "losa_within_lvsa_720p": lvsa_losa,
         "lvsa_build_index": {"us": index_us, "bytes_out": (wl.T * wl.T + wl.T) * 4,
                              "note": "a few KB written: latency-bound, GB/s not meaningful"},
         "context_torch_sdpa_dense": sdpa,
@@ -439,6 +441,59 @@ def run_sdpa_context(qkv, scale, stream, reps=2):
         return {"ms": statistics.median(ms), "tflops": 4 * d * H * N * N / (statistics.median(ms) / 1e3) / 1e12}
     except Exception as e:                                        # noqa: BLE001 - context only
         return {"unavailable": str(e).splitlines()[0][:200]}
+
+
+def run_lvsa_losa(bsa, stream, heads=4):
+    """LoSA's selection inside LVSA's frame sets on the 720p Wan-14B shape
+    (T=63 x P=3600, d=128), `heads` of its 40 heads: the restricted measuring
+    step (LVSA attention + block mass), the selection, and a later step on
+    the intersection index against LVSA alone.  Times scale with heads."""
+    import dataclasses
+    wl = dataclasses.replace(WORKLOADS["720p_14b"], H=heads)
+    N, H, d, nB = wl.N, wl.H, wl.d, math.ceil(wl.N / 128)
+    q, k, v = inputs.workload_qkv(wl, 0, device="cuda")
+    frames, counts, _ = bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, 0, device="cuda")
+    ix = bsa.lvsa_index(wl.T, frames, counts)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, N), dtype=torch.float32, device="cuda")
+    mass = torch.empty((H, nB, nB), dtype=torch.float32, device="cuda")
+    ws_m = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKMASS, N, H, d, ix), dtype=torch.uint8, device="cuda")
+
+    def timed(fn, reps=2):
+        out = []
+        for i in range(reps + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i:
+                out.append(a.elapsed_time(b))
+        return statistics.median(out)
+
+    t_mass = timed(lambda: bsa.attn_blockmass(q, k, v, ix, wl.scale, o=o, lse=lse, mass=mass, workspace=ws_m,
+                                              stream=stream))
+    del ws_m
+    idx, cnt = bsa.losa_select(mass, wl.tau)
+    t_sel = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 10)
+    ix3 = bsa.lvsa_block_index(wl.T, frames, counts, idx, cnt)
+    ws_f = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix3), dtype=torch.uint8,
+                       device="cuda")
+    t_lvsa = timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, ix, scale=wl.scale, o=o, lse=lse, workspace=ws_f,
+                                                    stream=stream))
+    _, tcnt, _, _ = bsa.lvsa_workspace_views(ws_f, N, wl.T)
+    lvsa_tiles = int(tcnt.sum().item()) * H
+    t_both = timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, ix3, scale=wl.scale, o=o, lse=lse, workspace=ws_f,
+                                                    stream=stream))
+    status = bsa.get_device_status()
+    kept = int(cnt.sum().item())
+    flop = lambda tiles: 4 * d * tiles * 128 * 128               # noqa: E731
+    return {"workload": f"720p_14b: T=63 x P=3600 (N={N}), {H} of 40 heads, d=128, LVSA C=21 W=15 T_per=6, "
+                        "LoSA tau=0.99 inside the LVSA sets",
+            "restricted_mass_ms": t_mass, "select_us": t_sel * 1e3,
+            "lvsa_ms": t_lvsa, "lvsa_tflops_kept_tiles": flop(lvsa_tiles) / (t_lvsa / 1e3) / 1e12,
+            "intersection_ms": t_both, "intersection_tflops_kept_tiles": flop(kept) / (t_both / 1e3) / 1e12,
+            "kept_fraction_of_lvsa_tiles": kept / lvsa_tiles, "status": bsa.status_string(status)}
 
 
 def run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws, calls=6):
