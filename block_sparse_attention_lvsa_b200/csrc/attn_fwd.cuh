@@ -1,5 +1,6 @@
 // attn_fwd.cuh - block-sparse / dense softmax attention forward on sm_100a
-// tensor cores (tcgen05 + TMEM + TMA), and the LoSA block-mass pass.
+// tensor cores (tcgen05 + TMEM + TMA), with a mode that also records what
+// the LoSA block mass needs.
 //
 // Sources: "LVSA: Training-Free Sparse Attention for Long Video Diffusion"
 // (gist.science explainer), technical summary section 2 (block-sparse
@@ -40,13 +41,15 @@
 // packs P over the same registers.  Tiles flagged partial (frame boundary or
 // sequence end) get an element mask from the frame bit matrix.
 //
-// Mass mode (MASS = true) is the dense measuring step of LoSA in one pass:
-// the same forward, which also writes, per query row and key tile, the log2
-// of that tile's share of the row's probability mass before normalisation,
+// Mass mode (MASS = true) is LoSA's measuring step in one pass, on the dense
+// index or any other: the same forward, which also writes, per query row
+// and visited key tile, the log2 of that tile's share of the row's
+// probability mass before normalisation,
 // lpart = log2(sum_k exp2(s_k * scale * log2e - m)) + m with the stabiliser m
-// the row used for the tile.  The block mass of a (query block, key block)
-// pair is then sum over the block's rows of exp2(lpart - lse * log2e), which
-// a separate reduction forms once the final LSE is known.
+// the row used for the tile (tiles the index never reaches are not
+// written).  The block mass of a (query block, key block) pair is then the
+// sum over the block's rows of exp2(lpart - lse * log2e), which a separate
+// reduction forms once the final LSE is known.
 #pragma once
 #include "ptx.cuh"
 
