@@ -399,7 +399,7 @@ def run_b200(args, rank, world, local):
 # (656.4 MB read + 197.3 MB written, step-0 index) scaled by 12/4 - traffic
 # grows with the number of heads.  Must be re-measured (or set to None)
 # whenever the kernel changes.
-TRAFFIC_PER_LAUNCH = 2.561e9
+TRAFFIC_PER_LAUNCH = None
 
 
 def run_gather(o, lse, H, world, reps=3):

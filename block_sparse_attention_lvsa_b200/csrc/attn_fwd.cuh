@@ -248,8 +248,51 @@ constexpr int kPolyCols = 0;
 // exp2(s * sl2 - m) for one 128-score row; P (bf16 pairs) packed in place
 // into sr[0..63] (pair j overwrites sr[j] only after elements 2j, 2j+1 >= j
 // are read).  Returns the row sum of the float32 values.
+// Packed float pairs (Blackwell f32x2 FMA-pipe ops): one instruction does two
+// fmaf / two float adds with the same per-lane rounding.  The softmax uses
+// them for the score scaling and the row sums, halving its FMA-pipe
+// instructions; the pipe is shared with the MMA-issuing thread's
+// sub-partition, where FMA-dense code slows the issue of tensor-core work.
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 template <int NPOLY>
 __device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use) {
+  if constexpr (NPOLY == 0) {
+    const uint64_t sl2p = f2pack(sl2, sl2), nm = f2pack(-m_use, -m_use);
+    uint64_t acc01 = f2pack(0.f, 0.f), acc23 = f2pack(0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < 128; c += 4) {
+      float x0, x1, x2, x3;
+      f2unpack(ffma2(f2pack(s[c], s[c + 1]), sl2p, nm), x0, x1);
+      f2unpack(ffma2(f2pack(s[c + 2], s[c + 3]), sl2p, nm), x2, x3);
+      const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+      acc01 = fadd2(acc01, f2pack(e0, e1));
+      acc23 = fadd2(acc23, f2pack(e2, e3));
+      sr[c / 2] = pack_bf16x2(e0, e1);
+      sr[c / 2 + 1] = pack_bf16x2(e2, e3);
+    }
+    float r0, r1, r2, r3;
+    f2unpack(acc01, r0, r1);
+    f2unpack(acc23, r2, r3);
+    return (r0 + r1) + (r2 + r3);
+  }
   float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
 #pragma unroll
   for (int c = 0; c < 128; c += 4) {
