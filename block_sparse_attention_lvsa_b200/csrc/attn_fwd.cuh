@@ -16,11 +16,14 @@
 //
 // Warp roles (384 threads):
 //   warp 0       TMA producer: Q_0, Q_1 once, then K tiles (2-deep ring)
-//   warp 1       TMEM allocator and single-thread tcgen05.mma issuer
-//   warp 2       TMA producer: V tiles (3-deep ring; forward only)
+//   warp 1       TMEM allocator and tcgen05.mma issuer (the whole warp runs
+//                the loop, an elected lane issues)
+//   warp 2       TMA producer: V tiles (3-deep ring)
 //   warp 3       idle
 //   warps 4..7   softmax group 0: thread r owns row r of query tile 0
 //   warps 8..11  softmax group 1: thread r owns row r of query tile 1
+// setmaxnreg moves registers from warps 0..3 (72 each) to the softmax
+// warps (216 each), which hold a row's 128 scores in registers.
 // TMEM columns: S_0 [0,128), S_1 [128,256) (f32 scores), O_0 [256,256+d),
 // O_1 [256+d, 256+2d) (f32 accumulators).  The softmax writes P (bf16, two
 // per 32-bit column) over the first 64 columns of its S tile and the PV
@@ -83,6 +86,13 @@ constexpr int kQTilesPerCta = 2;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kKStages = 2;                        // K ring depth (128-key tiles)
 constexpr int kVStages = 3;                        // V ring depth (a V tile lives until O_1's PV)
+// setmaxnreg budgets (0 = off): warps 0..3 (producers, issuer, idle) and
+// the two softmax warpgroups; at most the launch's 168 x 384 registers.
+// Without the split the softmax spills ~100 bytes per thread inside its
+// tile loop; measured 44.2 -> 40.0 ms per headline call with it.
+constexpr int kRegsLow = 72;
+constexpr int kRegsHigh = 216;
+static_assert(kRegsLow * 128 + kRegsHigh * 256 <= 168 * kAttnThreads, "register split");
 
 template <int D, bool MASS>
 struct AttnSmem {
@@ -235,14 +245,12 @@ __device__ __forceinline__ float exp2_poly3(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
-// Of every 8 columns of an unmasked tile, kPolyCols / 16 take exp2_poly3 on
-// the FMA pipe and the rest ex2 on MUFU (masked tiles stay on MUFU: the
-// polynomial does not give exactly 0 for a masked score).  Off: FMA-dense
-// code in a softmax warp that shares a sub-partition with the MMA-issuing
-// thread slows the issue of every tcgen05.mma (measured: 64 -> ~120 cycles
-// per 128x128x16 MMA next to a warp issuing an FFMA per cycle), and every
-// sub-partition holds softmax warps; 16, 32 and 48 columns measured 10-20%
-// slower overall.
+// Of every 8 column pairs of an unmasked tile, kPolyCols / 16 take
+// exp2_poly3 on the FMA pipe and the rest ex2 on MUFU (masked tiles stay on
+// MUFU: the polynomial does not give exactly 0 for a masked score).  Off:
+// with the warp-wide MMA issue and the register split, 16 and 32 columns
+// measured the same as 0 (39.68 / 39.65 vs 39.70 ms): a softmax warp's
+// exponential phase is bound by its own instruction stream, not by MUFU.
 constexpr int kPolyCols = 0;
 
 // exp2(s * sl2 - m) for one 128-score row; P (bf16 pairs) packed in place
@@ -272,44 +280,81 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// exp2_poly3 on a packed pair: the adds and the polynomial run as f32x2
+// instructions (same per-lane rounding), the clamp and the exponent-field
+// add per lane.
+__device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t xp) {
+  float a, b;
+  f2unpack(xp, a, b);
+  xp = f2pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
+  const uint64_t t = fadd2(xp, f2pack(12582912.0f, 12582912.0f));
+  const uint64_t j = fadd2(t, f2pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = ffma2(j, f2pack(-1.0f, -1.0f), xp);
+  uint64_t q = ffma2(f2pack(0.0551716685295105f, 0.0551716685295105f), f,
+                     f2pack(0.2426111251115799f, 0.2426111251115799f));
+  q = ffma2(q, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
+  q = ffma2(q, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  float q0, q1, t0, t1;
+  f2unpack(q, q0, q1);
+  f2unpack(t, t0, t1);
+  return f2pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
+// column pair j (columns 2j, 2j+1) of an unmasked tile takes the polynomial:
+// NPOLY / 16 of every 8 pairs
 template <int NPOLY>
-__device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use) {
-  if constexpr (NPOLY == 0) {
-    const uint64_t sl2p = f2pack(sl2, sl2), nm = f2pack(-m_use, -m_use);
-    uint64_t acc01 = f2pack(0.f, 0.f), acc23 = f2pack(0.f, 0.f);
-#pragma unroll
-    for (int c = 0; c < 128; c += 4) {
-      float x0, x1, x2, x3;
-      f2unpack(ffma2(f2pack(s[c], s[c + 1]), sl2p, nm), x0, x1);
-      f2unpack(ffma2(f2pack(s[c + 2], s[c + 3]), sl2p, nm), x2, x3);
-      const float e0 = ex2_approx(x0), e1 = ex2_approx(x1), e2 = ex2_approx(x2), e3 = ex2_approx(x3);
-      acc01 = fadd2(acc01, f2pack(e0, e1));
-      acc23 = fadd2(acc23, f2pack(e2, e3));
-      sr[c / 2] = pack_bf16x2(e0, e1);
-      sr[c / 2 + 1] = pack_bf16x2(e2, e3);
-    }
-    float r0, r1, r2, r3;
-    f2unpack(acc01, r0, r1);
-    f2unpack(acc23, r2, r3);
-    return (r0 + r1) + (r2 + r3);
-  }
-  float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+__device__ __forceinline__ constexpr bool poly_pair(int j) {
+  return (j & 7) < NPOLY / 16;
+}
+
+// P of keys 0..63 (sr[0..31]) goes to TMEM as soon as it is formed, keys
+// 64..127 after the loop; the caller waits for both stores
+// (tmem_wait_st) before signalling P ready.
+constexpr bool kSplitPStore = true;
+
+template <int NPOLY>
+__device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use, uint32_t tP) {
+  const uint64_t sl2p = f2pack(sl2, sl2), nm = f2pack(-m_use, -m_use);
+  uint64_t acc01 = f2pack(0.f, 0.f), acc23 = f2pack(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 128; c += 4) {
-    float e[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float xx = fmaf(s[c + u], sl2, -m_use);
-      e[u] = (((c + u) & 7) * 16 < NPOLY) ? exp2_poly3(xx) : ex2_approx(xx);
+    const uint64_t x01 = ffma2(f2pack(s[c], s[c + 1]), sl2p, nm);
+    const uint64_t x23 = ffma2(f2pack(s[c + 2], s[c + 3]), sl2p, nm);
+    uint64_t e01, e23;
+    if (poly_pair<NPOLY>(c / 2)) {
+      e01 = exp2_poly3_x2(x01);
+    } else {
+      float x0, x1;
+      f2unpack(x01, x0, x1);
+      e01 = f2pack(ex2_approx(x0), ex2_approx(x1));
     }
-    rs0 += e[0];
-    rs1 += e[1];
-    rs2 += e[2];
-    rs3 += e[3];
-    sr[c / 2] = pack_bf16x2(e[0], e[1]);
-    sr[c / 2 + 1] = pack_bf16x2(e[2], e[3]);
+    if (poly_pair<NPOLY>(c / 2 + 1)) {
+      e23 = exp2_poly3_x2(x23);
+    } else {
+      float x2, x3;
+      f2unpack(x23, x2, x3);
+      e23 = f2pack(ex2_approx(x2), ex2_approx(x3));
+    }
+    acc01 = fadd2(acc01, e01);
+    acc23 = fadd2(acc23, e23);
+    float e0, e1, e2, e3;
+    f2unpack(e01, e0, e1);
+    f2unpack(e23, e2, e3);
+    sr[c / 2] = pack_bf16x2(e0, e1);
+    sr[c / 2 + 1] = pack_bf16x2(e2, e3);
+    if (kSplitPStore && c == 60) tmem_st_x32_async(tP, sr);
   }
-  return (rs0 + rs1) + (rs2 + rs3);
+  if (kSplitPStore) {
+    tmem_st_x32_async(tP + 32, sr + 32);
+  } else {
+    tmem_st_x32_async(tP, sr);
+    tmem_st_x32_async(tP + 32, sr + 32);
+  }
+  float r0, r1, r2, r3;
+  f2unpack(acc01, r0, r1);
+  f2unpack(acc23, r2, r3);
+  return (r0 + r1) + (r2 + r3);
 }
 
 template <int D, bool MASS>
@@ -393,6 +438,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (warp == 0) {
     // ============================================ TMA producer: Q, K ====
+    if constexpr (kRegsLow > 0) regs_dec<kRegsLow>();
     if (lane == 0 && any_work) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -421,6 +467,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else if (warp == 2) {
     // ============================================== TMA producer: V ====
+    if constexpr (kRegsLow > 0) regs_dec<kRegsLow>();
     if (lane == 0 && any_work) {
       tma_prefetch_desc(&tmV);
       int it = 0, kt;
@@ -440,44 +487,48 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else if (warp == 1) {
     // ================================================= MMA issuer ======
-    if (lane == 0 && any_work) {
+    if constexpr (kRegsLow > 0) regs_dec<kRegsLow>();
+    // The whole warp walks the lists and waits; one elected lane issues
+    // (see mma4_ss_warp for why the issue is not done from a lane-0 branch).
+    if (any_work) {
       bool ok = true, bad = false;
-      const SmemDesc dQ[2] = {sw128_desc(base + L::kQ, 16, 1024), sw128_desc(base + L::kQ + L::kTile, 16, 1024)};
+      const uint64_t dQ[2] = {desc64(sw128_desc(base + L::kQ, 16, 1024)),
+                              desc64(sw128_desc(base + L::kQ + L::kTile, 16, 1024))};
       int cnt[2] = {0, 0};          // per query tile: key tiles processed
       int it = 0, kt;
       bool in[2];
 
-      // S = Q_x K^T into TMEM column block `sb` (forward: sb = x; mass mode:
-      // sb = 2x + buffer), completion signalled on SFULL + sb
-      auto qk = [&](int x, int sb, int ks) {
-        const SmemDesc dk = sw128_desc(base + L::kK + ks * L::kTile, 16, 1024);
+      // S = Q_x K^T into TMEM column block `sb`, completion on SFULL + sb
+      // (and, when given, on a second barrier)
+      auto qk = [&](int x, int sb, int ks, int bar2) {
+        const uint64_t dk = desc64(sw128_desc(base + L::kK + ks * L::kTile, 16, 1024));
         const uint32_t dS = tbase + sb * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {     // 16 channels per step
-          const uint32_t off = ((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(dS, dQ[x].lo + off, dQ[x].hi, dk.lo + off, dk.hi, kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(B_SFULL + sb));
+        for (int g = 0; g < D / 64; ++g)          // 64 channels (one 128-byte box) per group of 4
+          mma4_ss_warp(dS, dQ[x] + g * (L::kBox >> 4), dk + g * (L::kBox >> 4), kIdescQK, g > 0 ? 1u : 0u);
+        if (bar2 >= 0) tc_commit2_warp(bar(B_SFULL + sb), bar(bar2));
+        else tc_commit_warp(bar(B_SFULL + sb));
       };
       // wait until V of key tile `vit` and P_x of the group's c-th tile are in place
       auto pv_ready = [&](int x, int vit, int c) -> bool {
-        if (!mbar_wait(bar(B_VFULL + vit % kVStages), (vit / kVStages) & 1, limit)) return false;
-        if (!mbar_wait(bar(B_PFULL + x), c & 1, limit)) return false;
+        if (!mbar_wait_warp(bar(B_VFULL + vit % kVStages), (vit / kVStages) & 1, limit)) return false;
+        if (!mbar_wait_warp(bar(B_PFULL + x), c & 1, limit)) return false;
         tc_fence_after();
         return true;
       };
-      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major)
-      auto pv = [&](int x, int vit, int c) {
-        const SmemDesc dv = sw128_desc(base + L::kV + (vit % kVStages) * L::kTile, L::kBox, 1024);
+      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major); completion
+      // on PVDONE + x (and, when given, on a second barrier)
+      auto pv = [&](int x, int vit, int c, int bar2) {
+        const uint64_t dv = desc64(sw128_desc(base + L::kV + (vit % kVStages) * L::kTile, L::kBox, 1024));
         const uint32_t tO = tbase + L::kTmemO + x * D;
         const uint32_t tP = tbase + x * 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)            // 16 keys per step: 8 TMEM columns of P, 2 KB of V
-          mma_bf16_ts(tO, tP + kk * 8, dv.lo + kk * 128, dv.hi, kIdescPV, (c > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_PVDONE + x));
+        mma4_ts_warp(tO, tP, dv, kIdescPV, c > 0 ? 1u : 0u);     // keys 0..63
+        mma4_ts_warp(tO, tP + 32, dv + 512, kIdescPV, 1u);       // keys 64..127
+        if (bar2 >= 0) tc_commit2_warp(bar(B_PVDONE + x), bar(bar2));
+        else tc_commit_warp(bar(B_PVDONE + x));
       };
 
-      if (!mbar_wait(bar(B_QFULL), 0, limit)) ok = false;
+      if (!mbar_wait_warp(bar(B_QFULL), 0, limit)) ok = false;
       tc_fence_after();
       {
         // Issue order per key tile i: O_1 += P_1(i-1) V, S_1(i), [next tile
@@ -490,36 +541,34 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         int pend_it = -1, pend_c = 0;       // O_1's PV of an earlier tile, not yet issued
         bool have = ok && pl.next(kt, in, bad);
         if (have) {
-          ok = mbar_wait(bar(B_KFULL), 0, limit);
+          ok = mbar_wait_warp(bar(B_KFULL), 0, limit);
           tc_fence_after();
-          if (ok && in[0]) qk(0, 0, 0);
+          if (ok && in[0]) qk(0, 0, 0, -1);
         }
         while (ok && have) {
           const int ks = it % kKStages;
           if (pend_it >= 0) {
             ok = pv_ready(1, pend_it, pend_c);
             if (!ok) break;
-            pv(1, pend_it, pend_c);
-            tc_commit(bar(B_VEMPTY + pend_it % kVStages));
+            pv(1, pend_it, pend_c, B_VEMPTY + pend_it % kVStages);
             pend_it = -1;
           }
-          if (in[1]) qk(1, 1, ks);
-          tc_commit(bar(B_KEMPTY + ks));
+          if (in[1]) qk(1, 1, ks, B_KEMPTY + ks);
+          else tc_commit_warp(bar(B_KEMPTY + ks));
           int nkt = 0;
           bool nin[2] = {false, false};
           const bool nhave = pl.next(nkt, nin, bad);
           if (nhave) {
-            ok = mbar_wait(bar(B_KFULL + (it + 1) % kKStages), ((it + 1) / kKStages) & 1, limit);
+            ok = mbar_wait_warp(bar(B_KFULL + (it + 1) % kKStages), ((it + 1) / kKStages) & 1, limit);
             if (!ok) break;
             tc_fence_after();
           }
           if (in[0]) {
             ok = pv_ready(0, it, cnt[0]);
             if (!ok) break;
-            pv(0, it, cnt[0]);
-            if (!in[1]) tc_commit(bar(B_VEMPTY + it % kVStages));
+            pv(0, it, cnt[0], in[1] ? -1 : B_VEMPTY + it % kVStages);
           }
-          if (nhave && nin[0]) qk(0, 0, (it + 1) % kKStages);
+          if (nhave && nin[0]) qk(0, 0, (it + 1) % kKStages, -1);
           if (in[1]) {
             pend_it = it;
             pend_c = cnt[1];
@@ -532,18 +581,18 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           in[1] = nin[1];
           have = nhave;
         }
-        if (ok && pend_it >= 0 && pv_ready(1, pend_it, pend_c)) {
-          pv(1, pend_it, pend_c);
-          tc_commit(bar(B_VEMPTY + pend_it % kVStages));
-        }
+        if (ok && pend_it >= 0 && pv_ready(1, pend_it, pend_c)) pv(1, pend_it, pend_c, B_VEMPTY + pend_it % kVStages);
       }
-      if (bad) set_status(BSA_ERR_INDEX_RANGE);
+      if (bad && lane == 0) set_status(BSA_ERR_INDEX_RANGE);
       // all issued MMAs complete before the CTA may release TMEM
-      tc_commit(bar(B_FINAL));
-      mbar_wait(bar(B_FINAL), 0, limit);
+      tc_commit_warp(bar(B_FINAL));
+      mbar_wait_warp(bar(B_FINAL), 0, limit);
     }
+  } else if (warp == 3) {
+    if constexpr (kRegsLow > 0) regs_dec<kRegsLow>();   // idle: its registers go to the softmax warps
   } else if (warp >= 4) {
     // ================================================= softmax groups ==
+    if constexpr (kRegsLow > 0) regs_inc<kRegsHigh>();
     const int x = (threadIdx.x - 128) >> 7;           // query tile 0 or 1 of this CTA
     const int r = (threadIdx.x - 128) & 127;          // row within the tile = TMEM lane
     const int qt = qt0 + x;
@@ -612,8 +661,9 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         // p = exp2(s * scale * log2e - m), P packed in place (the tile's flag is
         // the same for the whole group: no divergence)
-        const float rsum = part ? row_exp_pack<0>(s, sr, p.sl2, m_use) : row_exp_pack<kPolyCols>(s, sr, p.sl2, m_use);
-        tmem_st_x64(tS, sr);
+        const float rsum =
+            part ? row_exp_pack<0>(s, sr, p.sl2, m_use, tS) : row_exp_pack<kPolyCols>(s, sr, p.sl2, m_use, tS);
+        tmem_wait_st();
         if constexpr (MASS) {
           // this tile's share of the row's mass, log2, before normalisation
           if (q < p.N)

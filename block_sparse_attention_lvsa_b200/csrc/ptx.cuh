@@ -158,6 +158,73 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Warp-wide issue: the whole (converged) warp executes these, one elected
+// lane issues.  Four MMAs and the commits share one elect, and the operand
+// descriptors are whole 64-bit values advanced by immediates inside the asm
+// block.  A thread issuing alone from a lane-0 branch, next to a warp that
+// issues an FMA-pipe instruction every cycle on the same sub-partition,
+// measured ~120 cycles per 128x128x16 MMA; this form measured 66 (64 with
+// no neighbour).  The same lane (the lowest) is elected every time, so the
+// commits track the MMAs that lane issued.
+//
+// D[tmem] (+)= A[smem] * B[smem]^T for four consecutive K-steps of 16
+// (descriptor start address + 32 B each, SW128 K-major operands).
+__device__ __forceinline__ void mma4_ss_warp(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                             uint32_t accumulate_first) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, b1;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 t, %5, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 a1, %1, 2;\n\tadd.s64 b1, %2, 2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+      "add.s64 a1, %1, 4;\n\tadd.s64 b1, %2, 4;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t"
+      "add.s64 a1, %1, 6;\n\tadd.s64 b1, %2, 6;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a1, b1, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate_first), "r"(1u)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem] for four consecutive K-steps of 16: A moves
+// 8 TMEM columns (16 bf16) and B (MN-major, 128-byte rows) 2 KB per step.
+__device__ __forceinline__ void mma4_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                             uint32_t accumulate_first) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, t;\n\t.reg .b64 b1;\n\t.reg .b32 a1;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 t, %5, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.u32 a1, %1, 8;\n\tadd.s64 b1, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+      "add.u32 a1, %1, 16;\n\tadd.s64 b1, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+      "add.u32 a1, %1, 24;\n\tadd.s64 b1, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate_first), "r"(1u)
+      : "memory");
+}
+// commit of the elected lane's MMAs to one barrier, or to two
+__device__ __forceinline__ void tc_commit_warp(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit2_warp(uint32_t bar0, uint32_t bar1) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%1];\n\t}" ::"r"(bar0),
+      "r"(bar1)
+      : "memory");
+}
+// bounded wait with a warp-uniform result (every lane polls the barrier)
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, long long limit_ns) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, limit_ns));
+}
+
 // UMMA shared-memory descriptor of a 128-byte-swizzled operand, split in
 // 32-bit halves: lo = start address >> 4 | leading byte offset >> 4 << 16,
 // hi = stride byte offset >> 4 | version 1 << 14 | SWIZZLE_128B (2) << 29.
@@ -171,6 +238,9 @@ __device__ __forceinline__ SmemDesc sw128_desc(uint32_t saddr, uint32_t lbo_byte
   d.lo = ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
   d.hi = ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
   return d;
+}
+__device__ __forceinline__ uint64_t desc64(SmemDesc d) {
+  return (static_cast<uint64_t>(d.hi) << 32) | d.lo;
 }
 
 // Instruction descriptor: bf16 x bf16 -> f32, M x N tile, operand majors.
@@ -231,6 +301,28 @@ __device__ __forceinline__ void tmem_st_x64(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};\n\t"
                "tcgen05.wait::st.sync.aligned;"
                :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63]) : "memory");
+}
+
+// Store without waiting: the registers may be reused only after
+// tmem_wait_st() (which waits for every earlier store of the thread).
+__device__ __forceinline__ void tmem_st_x32_async(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]) : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Per-warpgroup register budget (every warp of a warpgroup executes the same
+// instruction).  .inc waits until registers released by .dec exist, so the
+// budgets must add up to at most the block's registers at launch.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
