@@ -396,10 +396,10 @@ def run_b200(args, rank, world, local):
 
 # DRAM bytes (read + write) per launch of the attention kernel at the full
 # 12-head workload: the ncu capture of the 4-head case of the same workload
-# (645.8 MB read + 195.9 MB written, step-0 index) scaled by 12/4 - traffic
+# (658.5 MB read + 190.7 MB written, step-0 index) scaled by 12/4 - traffic
 # grows with the number of heads.  Must be re-measured (or set to None)
 # whenever the kernel changes.
-TRAFFIC_PER_LAUNCH = 2.525e9
+TRAFFIC_PER_LAUNCH = 2.548e9
 
 
 def run_gather(o, lse, H, world, reps=3):
