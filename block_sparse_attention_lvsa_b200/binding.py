@@ -79,7 +79,7 @@ def _load():
         "bsa_workspace_bytes": (SZ, [I, I, I, I, ctypes.POINTER(bsa_index)]),
         "bsa_get_device_status": (I, [P]),
         "bsa_status_string": (ctypes.c_char_p, [I]),
-        "bsa_debug_expired_wait": (I, [ctypes.c_longlong, P]),
+        "bsa_debug_expired_wait": (I, [ctypes.c_longlong, I, P]),
         "bsa_version": (ctypes.c_char_p, []),
         "blocksparse_attn_fwd_noalloc": (I, [P, P, P, I, I, I, F, ctypes.POINTER(bsa_index), P, P, P]),
     }
@@ -308,8 +308,9 @@ def get_device_status(stream=None) -> int:
     return int(_lib.bsa_get_device_status(_stream(stream)))
 
 
-def debug_expired_wait(limit_ns: int, stream=None) -> int:
-    return int(_lib.bsa_debug_expired_wait(int(limit_ns), _stream(stream)))
+def debug_expired_wait(limit_ns: int, form: int = 0, stream=None) -> int:
+    """Enqueue the expired-wait diagnostic (form 0: one thread waits, 1: the whole warp)."""
+    return int(_lib.bsa_debug_expired_wait(int(limit_ns), int(form), _stream(stream)))
 
 
 def lvsa_workspace_views(workspace: torch.Tensor, N: int, T: int):

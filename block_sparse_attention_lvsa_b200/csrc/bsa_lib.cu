@@ -391,21 +391,28 @@ int bsa_get_device_status(void* stream) {
 }  // extern "C"
 
 namespace {
-__global__ void debug_expired_wait_kernel(long long limit_ns) {
+__global__ void debug_expired_wait_kernel(long long limit_ns, int form) {
   __shared__ alignas(8) unsigned long long bar;
+  const uint32_t b = smem_u32(&bar);
   if (threadIdx.x == 0) {
-    const uint32_t b = smem_u32(&bar);
     mbar_init(b, 1);
     fence_mbar_init();
-    // nothing ever arrives on this barrier: the wait must give up by itself
-    mbar_wait(b, 0, limit_ns);
+  }
+  __syncthreads();
+  // nothing ever arrives on this barrier: the wait must give up by itself
+  if (form == 0) {
+    if (threadIdx.x == 0) mbar_wait(b, 0, limit_ns);
+  } else {
+    // the whole-warp form: every lane must see the same (false) result
+    const bool ok = mbar_wait_warp(b, 0, limit_ns);
+    if (__any_sync(0xFFFFFFFFu, ok) && threadIdx.x == 0) atomicExch(&g_bsa_status, BSA_ERR_ARG);
   }
 }
 }  // namespace
 
-extern "C" int bsa_debug_expired_wait(long long limit_ns, void* stream) {
-  if (limit_ns < 100000LL || limit_ns > 10000000000LL) return BSA_ERR_ARG;
-  debug_expired_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+extern "C" int bsa_debug_expired_wait(long long limit_ns, int form, void* stream) {
+  if (limit_ns < 100000LL || limit_ns > 10000000000LL || form < 0 || form > 1) return BSA_ERR_ARG;
+  debug_expired_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, form);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
 

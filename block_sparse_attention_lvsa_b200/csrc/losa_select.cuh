@@ -13,11 +13,14 @@
 // (Q desc, kb asc), the prefix is {kb : key_kb >= pivot}, where pivot is the
 // largest key x with S(x) = sum_{key >= x} Q >= threshold (S only drops at
 // keys, so that x is itself a key).  One warp per row finds the pivot by
-// bisection over the key bits: each step is a compare-and-sum over the row
-// and a 64-bit warp-shuffle reduction - no sorting, no atomics, no block
-// barriers.  The kept ids are then written in ascending kb order with warp
-// ballots.  Every sum is a 64-bit integer, so the result does not depend on
-// the order of accumulation.
+// bisection: each step is a compare-and-sum over the row and a 64-bit
+// warp-shuffle reduction - no sorting, no atomics, no block barriers.  Rows
+// of up to 2048 blocks (registers) bisect over the 31 bits of the mass
+// instead of the 57-bit keys and settle ties in Q by kb afterwards (see
+// losa_select_reg_kernel); longer rows (shared memory) bisect over the keys.
+// The kept ids are then written in ascending kb order with warp ballots.
+// Every sum is a 64-bit integer, so the result does not depend on the order
+// of accumulation.
 #pragma once
 #include "ptx.cuh"
 
@@ -101,10 +104,18 @@ __global__ void losa_select_kernel(const float* __restrict__ mass, int rows, int
   }
 }
 
-// Same computation with the row's keys in registers (nKB <= 32 * KPL): lane
-// l holds the keys of blocks l, l+32, ...; loads are unrolled, and the pivot
-// search decides two key bits per round (three candidate thresholds, three
-// independent warp reductions), halving the dependent rounds.
+// Same result with the row in registers (nKB <= 32 * KPL; lane l holds
+// blocks l, l+32, ...), found by a search over 32-bit values instead of the
+// 64-bit keys.  Q is a non-decreasing function of the mass, and the bit
+// pattern of a non-negative float orders like its value, so
+// S(u) = sum of Q over blocks whose mass bits are >= u is non-increasing in
+// u.  Bisection over the 31 bits gives the largest u with S(u) >= threshold;
+// u is the mass bits of some block, and its Q is the pivot value Qp.  Every
+// block with Q > Qp has a larger mass, so their Q-sum A stays below the
+// threshold (else u + 1 would qualify), and the kept set is every block
+// with Q > Qp plus the first ceil((threshold - A) / Qp) blocks with Q == Qp
+// in ascending kb order: the shortest prefix of the (Q desc, kb asc) order.
+// A zero threshold (all masses zero) keeps the first block of that order.
 template <int KPL>
 __global__ void losa_select_reg_kernel(const float* __restrict__ mass, int rows, int nKB, double tau,
                                        int32_t* __restrict__ idx, int32_t* __restrict__ cnt) {
@@ -112,14 +123,15 @@ __global__ void losa_select_reg_kernel(const float* __restrict__ mass, int rows,
   const int wpc = blockDim.x >> 5;
   for (int row = blockIdx.x * wpc + (threadIdx.x >> 5); row < rows; row += gridDim.x * wpc) {
     const float* m = mass + static_cast<size_t>(row) * nKB;
-    unsigned long long key[KPL];
+    unsigned long long q[KPL];
+    uint32_t mb[KPL];
     float mv[KPL];
 #pragma unroll
     for (int j = 0; j < KPL; ++j) {
       const int i = lane + 32 * j;
       mv[j] = (i < nKB) ? m[i] : 0.0f;
     }
-    unsigned long long total = 0, kmax = 0;
+    unsigned long long total = 0, qmax = 0;
     bool bad = false;
 #pragma unroll
     for (int j = 0; j < KPL; ++j) {
@@ -129,58 +141,53 @@ __global__ void losa_select_reg_kernel(const float* __restrict__ mass, int rows,
         bad = bad || (i < nKB);
         xv = (xv >= 16384.0f) ? 16383.999f : 0.0f;
       }
-      const unsigned long long q = static_cast<unsigned long long>(static_cast<double>(xv) * 8589934592.0);
-      // padding slots get key 0: below every real key (real keys carry 65535 - kb > 0)
-      key[j] = (i < nKB) ? ((q << 16) | static_cast<unsigned long long>(65535 - i)) : 0ull;
-      total += (i < nKB) ? q : 0ull;
-      kmax = key[j] > kmax ? key[j] : kmax;
+      // padding slots: Q = 0 and mass bits 0, never counted or kept
+      q[j] = (i < nKB) ? static_cast<unsigned long long>(static_cast<double>(xv) * 8589934592.0) : 0ull;
+      mb[j] = (i < nKB) ? (__float_as_uint(xv) & 0x7FFFFFFFu) : 0u;   // -0.0 orders as +0.0
+      total += q[j];
+      qmax = q[j] > qmax ? q[j] : qmax;
     }
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(BSA_ERR_ARG);
     total = warp_sum_u64(total);
-    kmax = warp_max_u64(kmax);
     const unsigned long long thr =
         static_cast<unsigned long long>(ceil(__dmul_rn(tau, __ull2double_rn(total))));
-    unsigned long long pivot = kmax;
-    if (thr > 0) {
-      unsigned long long prefix = 0;
-      int b = 63 - __clzll(static_cast<long long>(kmax));   // highest bit that can be set
-      if ((b & 1) == 0) {                                    // odd number of bits: one binary round
-        const unsigned long long c = 1ull << b;
-        unsigned long long s0 = 0;
+    unsigned long long qp, take;          // pivot value, blocks of Q == qp to keep
+    if (thr == 0) {
+      qp = warp_max_u64(qmax);
+      take = 1;
+    } else {
+      uint32_t u = 0;
+      for (int b = 30; b >= 0; --b) {
+        const uint32_t c = u | (1u << b);
+        unsigned long long sum = 0;
 #pragma unroll
-        for (int j = 0; j < KPL; ++j) s0 += (key[j] >= c) ? (key[j] >> 16) : 0ull;
-        if (warp_sum_u64(s0) >= thr) prefix = c;
-        --b;
+        for (int j = 0; j < KPL; ++j) sum += (mb[j] >= c) ? q[j] : 0ull;
+        if (warp_sum_u64(sum) >= thr) u = c;
       }
-      for (; b >= 1; b -= 2) {                               // bits b, b-1 per round
-        const unsigned long long c1 = prefix | (1ull << (b - 1));
-        const unsigned long long c2 = prefix | (2ull << (b - 1));
-        const unsigned long long c3 = prefix | (3ull << (b - 1));
-        unsigned long long s1 = 0, s2 = 0, s3 = 0;
+      unsigned long long qu = 0;
 #pragma unroll
-        for (int j = 0; j < KPL; ++j) {
-          const unsigned long long qj = key[j] >> 16;
-          s1 += (key[j] >= c1) ? qj : 0ull;
-          s2 += (key[j] >= c2) ? qj : 0ull;
-          s3 += (key[j] >= c3) ? qj : 0ull;
-        }
+      for (int j = 0; j < KPL; ++j) qu = (mb[j] == u && lane + 32 * j < nKB) ? q[j] : qu;
+      qp = warp_max_u64(qu);
+      unsigned long long above = 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
-          s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
-          s3 += __shfl_xor_sync(0xFFFFFFFFu, s3, o);
-        }
-        // S is non-increasing: take the largest candidate that still reaches thr
-        prefix = (s3 >= thr) ? c3 : (s2 >= thr) ? c2 : (s1 >= thr) ? c1 : prefix;
-      }
-      pivot = prefix;
+      for (int j = 0; j < KPL; ++j) above += (q[j] > qp) ? q[j] : 0ull;
+      above = warp_sum_u64(above);
+      // thr > above and qp >= 1 here (see above); the guards only keep a
+      // malformed row from dividing by zero
+      const unsigned long long need = thr > above ? thr - above : 1ull;
+      take = qp > 0 ? (need + qp - 1) / qp : 1ull;
     }
     int32_t* out = idx + static_cast<size_t>(row) * nKB;
     int running = 0;
+    unsigned long long ties = 0;
 #pragma unroll
     for (int j = 0; j < KPL; ++j) {
       const int i = lane + 32 * j;
-      const bool keep = (i < nKB) && (key[j] >= pivot);
+      const bool tie = (i < nKB) && (q[j] == qp);
+      const unsigned int tmask = __ballot_sync(0xFFFFFFFFu, tie);
+      const unsigned long long rank = ties + __popc(tmask & ((1u << lane) - 1u));
+      ties += __popc(tmask);
+      const bool keep = (i < nKB) && (q[j] > qp || (tie && rank < take));
       const unsigned int bmask = __ballot_sync(0xFFFFFFFFu, keep);
       if (keep) out[running + __popc(bmask & ((1u << lane) - 1u))] = i;
       running += __popc(bmask);

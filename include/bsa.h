@@ -323,14 +323,18 @@ const char* bsa_status_string(int status);
 
 /*
  * bsa_debug_expired_wait - diagnostic for the bounded-wait machinery.
- * Enqueues one tiny kernel whose single thread waits on a barrier that
- * nothing ever signals, giving up after 2 * `limit_ns` SM clock cycles
- * (`limit_ns` nanoseconds at 2 GHz; `limit_ns` in 1e5..1e10) and recording
- * BSA_ERR_TIMEOUT in the status word.  Lets tests check that
- * an expired wait ends the kernel and leaves the context usable.  No part
- * of the pages corresponds to it.
+ * Enqueues one tiny kernel (one warp) that waits on a barrier that nothing
+ * ever signals, giving up after 2 * `limit_ns` SM clock cycles (`limit_ns`
+ * nanoseconds at 2 GHz; `limit_ns` in 1e5..1e10) and recording
+ * BSA_ERR_TIMEOUT in the status word.  `form` 0: one thread waits (the
+ * producers' and softmax warps' form); 1: the whole warp waits and must get
+ * the same failed result in every lane (the MMA issuer's form; a lane that
+ * saw the wait succeed records BSA_ERR_ARG instead).  Lets tests check that
+ * an expired wait ends the kernel and leaves the context usable.  Returns
+ * BSA_ERR_ARG for an out-of-range `limit_ns` or `form`.  No part of the
+ * pages corresponds to it.
  */
-int bsa_debug_expired_wait(long long limit_ns, void* stream);
+int bsa_debug_expired_wait(long long limit_ns, int form, void* stream);
 
 /* bsa_version - library version string. */
 const char* bsa_version(void);

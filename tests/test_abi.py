@@ -139,4 +139,5 @@ def test_host_validation_rejects_before_launch(bsa):
     assert s(fake, 2, 4, 4, 0.0, fake, fake, nul) == bsa.BSA_ERR_ARG
     assert s(fake, 2, 4, 4, 1.5, fake, fake, nul) == bsa.BSA_ERR_ARG
     assert s(fake, 2, 4, 9000, 0.99, fake, fake, nul) == bsa.BSA_ERR_UNSUPPORTED
-    assert L.bsa_debug_expired_wait(10, nul) == bsa.BSA_ERR_ARG
+    assert L.bsa_debug_expired_wait(10, 0, nul) == bsa.BSA_ERR_ARG
+    assert L.bsa_debug_expired_wait(1_000_000, 2, nul) == bsa.BSA_ERR_ARG

@@ -128,6 +128,25 @@ def test_losa_select_random(bsa, nKB):
         assert np.array_equal(idx.cpu().numpy(), ref_idx), tau
 
 
+@pytest.mark.parametrize("nKB", [5, 256, 1772])
+def test_losa_select_q_collisions(bsa, nKB):
+    """Distinct masses below 2^-9 share Q = floor(mass * 2^33): the (Q desc, kb asc)
+    order must decide among them by kb, not by mass; -0.0 counts as zero."""
+    rng = np.random.default_rng(100 + nKB)
+    H, nQB = 2, 4
+    m = ((rng.integers(0, 4, (H, nQB, nKB)) + rng.random((H, nQB, nKB))) * 2.0 ** -33).astype(np.float32)
+    m[0, 1, :: 4] = 2.0 ** -20                                 # a few larger, tied masses
+    m[1, 2, 0] = 64.0                                          # one dominant block
+    m[1, 3, 1::2] = -0.0
+    mass = torch.from_numpy(m).cuda()
+    for tau in (0.99, 0.5, 1.0):
+        idx, cnt = bsa.losa_select(mass, tau)
+        assert bsa.get_device_status() == bsa.BSA_OK
+        ref_idx, ref_cnt = olosa.select(m, tau)
+        assert np.array_equal(cnt.cpu().numpy(), ref_cnt), tau
+        assert np.array_equal(idx.cpu().numpy(), ref_idx), tau
+
+
 def test_losa_select_rejects_bad_mass(bsa):
     m = torch.tensor([[[0.5, float("nan"), -1.0, 3.0]]], dtype=torch.float32, device="cuda")
     bsa.losa_select(m, 0.99)

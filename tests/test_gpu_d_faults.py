@@ -24,11 +24,13 @@ def small_call(bsa):
     return o
 
 
-def test_expired_wait_reports_timeout(bsa):
+@pytest.mark.parametrize("form", [0, 1])
+def test_expired_wait_reports_timeout(bsa, form):
+    """form 0: one thread waits; 1: the whole warp waits (the MMA issuer's form)."""
     assert bsa.get_device_status() == bsa.BSA_OK
-    assert bsa.debug_expired_wait(20_000_000) == bsa.BSA_OK     # 20 ms
+    assert bsa.debug_expired_wait(20_000_000, form) == bsa.BSA_OK   # 20 ms
     assert bsa.get_device_status() == bsa.BSA_ERR_TIMEOUT
-    o = small_call(bsa)                                          # context still usable
+    o = small_call(bsa)                                              # context still usable
     assert bsa.get_device_status() == bsa.BSA_OK
     assert torch.isfinite(o.float()).all()
 
