@@ -225,28 +225,8 @@ __device__ __forceinline__ void apply_mask128(float* s, const uint32_t (&mw)[4])
     if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
 }
 
-// 2^x on the FMA pipe, for x <= ~10 (inputs below -125 give ~2^-125, not 0;
-// the clamp keeps the exponent field of the result positive).
-// x = j + f with j = round(x) (adding and removing 1.5 * 2^23 rounds to the
-// nearest integer) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted
-// by Remez exchange for minimum relative error on [-1/2, 1/2] (max relative
-// error 7.5e-5, below the bf16 half-ulp of 2^-9 that P is rounded to); 2^j is
-// added to the exponent field as an integer.  Available to take part of the
-// exponentials of unmasked tiles off the MUFU unit (kPolyCols columns).
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float j = t - 12582912.0f;
-  const float f = x - j;
-  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  // the exponent of t's bit pattern cancels: (0x4B400000 << 23) == 0 mod 2^32
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 // Of every 8 column pairs of an unmasked tile, kPolyCols / 16 take
-// exp2_poly3 on the FMA pipe and the rest ex2 on MUFU (masked tiles stay on
+// exp2_poly3_x2 on the FMA pipe and the rest ex2 on MUFU (masked tiles stay on
 // MUFU: the polynomial does not give exactly 0 for a masked score).  Off:
 // with the warp-wide MMA issue and the register split, 16 and 32 columns
 // measured the same as 0 (39.68 / 39.65 vs 39.70 ms): a softmax warp's
@@ -280,9 +260,18 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// exp2_poly3 on a packed pair: the adds and the polynomial run as f32x2
-// instructions (same per-lane rounding), the clamp and the exponent-field
-// add per lane.
+// 2^x of a packed pair on the FMA pipe, for x <= ~10 (inputs below -125
+// give ~2^-125, not 0; the clamp keeps the exponent field of the result
+// positive).
+// x = j + f with j = round(x) (adding and removing 1.5 * 2^23 rounds to the
+// nearest integer) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted
+// by Remez exchange for minimum relative error on [-1/2, 1/2] (max relative
+// error 7.5e-5, below the bf16 half-ulp of 2^-9 that P is rounded to); 2^j is
+// added to the exponent field as an integer (the exponent of t's bit pattern
+// cancels: (0x4B400000 << 23) == 0 mod 2^32).  The adds and the polynomial
+// run as f32x2 instructions (same per-lane rounding), the clamp and the
+// exponent-field add per lane.  Available to take part of the exponentials
+// of unmasked tiles off the MUFU unit (kPolyCols columns).
 __device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t xp) {
   float a, b;
   f2unpack(xp, a, b);
