@@ -1,6 +1,7 @@
-"""The FMA-pipe exponential used for part of the softmax columns (CPU only).
+"""The FMA-pipe exponential available for part of the softmax columns (CPU only).
 
-Replays the kernel's float32 recipe (constants read from the CUDA source) and
+Replays the kernel's float32 recipe (exp2_poly3_x2: each lane of the packed
+pair takes the same steps; constants read from the CUDA source) and
 checks it against the exact 2^x: relative error below 1e-4 wherever 2^x is a
 normal float, a finite positive result everywhere (very negative inputs are
 clamped), and results far below every probability that matters for inputs
@@ -16,12 +17,13 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 def kernel_recipe():
     src = open(SRC).read()
-    body = src[src.index("exp2_poly3(float x) {"):]
+    body = src[src.index("exp2_poly3_x2(uint64_t xp) {"):]
     body = body[:body.index("\n}")]
-    clamp = float(re.search(r"fmaxf\(x, (-?[0-9.]+)f\)", body).group(1))
-    m = re.search(r"fmaf\(([0-9.]+)f, f, ([0-9.]+)f\)", body)
+    clamp = float(re.search(r"fmaxf\(a, (-?[0-9.]+)f\)", body).group(1))
+    pair = r"f2pack\(([0-9.]+)f, \1f\)"      # the same constant in both lanes
+    m = re.search(r"ffma2\(" + pair + r", f,\s*f2pack\(([0-9.]+)f, \2f\)\)", body)
     c3, c2 = float(m.group(1)), float(m.group(2))
-    c1, c0 = [float(v) for v in re.findall(r"fmaf\(p, f, ([0-9.]+)f\)", body)]
+    c1, c0 = [float(v) for v in re.findall(r"ffma2\(q, f, f2pack\(([0-9.]+)f, \1f\)\)", body)]
     f32 = np.float32
 
     def exp2(x):
