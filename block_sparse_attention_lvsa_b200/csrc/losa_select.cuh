@@ -33,6 +33,14 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
   return v;
 }
+// ceil(tau * (double)total) with one IEEE double multiply, never above the
+// total: for totals above 2^53 the conversion to double can round up, and a
+// threshold the whole row cannot reach would make the kept set ill-defined
+// (the shortest prefix reaching the total is then the answer).
+__device__ __forceinline__ unsigned long long select_threshold(double tau, unsigned long long total) {
+  const unsigned long long t = static_cast<unsigned long long>(ceil(__dmul_rn(tau, __ull2double_rn(total))));
+  return t < total ? t : total;
+}
 __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -71,8 +79,7 @@ __global__ void losa_select_kernel(const float* __restrict__ mass, int rows, int
     total = warp_sum_u64(total);
     kmax = warp_max_u64(kmax);
     __syncwarp();
-    const unsigned long long thr =
-        static_cast<unsigned long long>(ceil(__dmul_rn(tau, __ull2double_rn(total))));
+    const unsigned long long thr = select_threshold(tau, total);
     // 2. pivot = largest key x with S(x) >= thr (thr == 0: the largest key)
     unsigned long long pivot = kmax;
     if (thr > 0) {
@@ -149,8 +156,7 @@ __global__ void losa_select_reg_kernel(const float* __restrict__ mass, int rows,
     }
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(BSA_ERR_ARG);
     total = warp_sum_u64(total);
-    const unsigned long long thr =
-        static_cast<unsigned long long>(ceil(__dmul_rn(tau, __ull2double_rn(total))));
+    const unsigned long long thr = select_threshold(tau, total);
     unsigned long long qp, take;          // pivot value, blocks of Q == qp to keep
     if (thr == 0) {
       qp = warp_max_u64(qmax);

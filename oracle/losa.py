@@ -11,7 +11,9 @@ The algorithm, step by step, per (head, query block) row of block masses:
      (exact: float32 -> float64 -> scale by a power of two -> floor);
   2. order the key blocks by Q descending, equal Q by key-block id ascending;
   3. total = sum of Q;  threshold = ceil(tau * total) with one IEEE float64
-     multiply (tau * float64(total));
+     multiply (tau * float64(total)), and never more than the total (a row
+     total above 2**53 can round up when converted to float64; the kept set
+     holds at least the fraction tau, so it needs at most the whole row);
   4. keep the shortest prefix of the order whose running sum of Q reaches the
      threshold (at least one block);
   5. emit the kept key-block ids in ascending order.
@@ -53,7 +55,7 @@ def select_row(mass_row, tau: float) -> List[int]:
         return []
     order = sorted(range(n), key=lambda kb: (-Q[kb], kb))
     total = sum(Q)
-    threshold = math.ceil(tau * float(total))
+    threshold = min(math.ceil(tau * float(total)), total)
     running = 0
     k = n
     for i, kb in enumerate(order):
@@ -97,6 +99,6 @@ def select_row_fast(mass_row, tau: float) -> np.ndarray:
     order = np.lexsort((kb, -Q))                 # Q desc, then kb asc
     run = np.cumsum(Q[order])
     total = int(run[-1])
-    threshold = math.ceil(tau * float(total))
+    threshold = min(math.ceil(tau * float(total)), total)
     k = int(np.argmax(run >= threshold)) + 1
     return np.sort(order[:k]).astype(np.int32)

@@ -147,6 +147,23 @@ def test_losa_select_q_collisions(bsa, nKB):
         assert np.array_equal(idx.cpu().numpy(), ref_idx), tau
 
 
+@pytest.mark.parametrize("n_zero", [0, 43, 2000])
+def test_losa_select_large_total(bsa, n_zero):
+    """Row totals above 2^53 whose float64 conversion rounds up (the threshold is
+    clamped to the total): the register kernel (<= 2048 blocks) and the
+    shared-memory kernel (longer rows) must both keep exactly the oracle's set."""
+    from tests.test_oracle_losa import large_total_row
+    row = large_total_row(n_zero)
+    m = np.stack([row, row[::-1].copy()])[None]              # [1, 2, nKB]
+    mass = torch.from_numpy(np.ascontiguousarray(m)).cuda()
+    for tau in (1.0, 0.99):
+        idx, cnt = bsa.losa_select(mass, tau)
+        assert bsa.get_device_status() == bsa.BSA_OK
+        ref_idx, ref_cnt = olosa.select(m, tau)
+        assert np.array_equal(cnt.cpu().numpy(), ref_cnt), tau
+        assert np.array_equal(idx.cpu().numpy(), ref_idx), tau
+
+
 def test_losa_select_rejects_bad_mass(bsa):
     m = torch.tensor([[[0.5, float("nan"), -1.0, 3.0]]], dtype=torch.float32, device="cuda")
     bsa.losa_select(m, 0.99)
