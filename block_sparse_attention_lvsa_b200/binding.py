@@ -131,12 +131,50 @@ def _check_qkv(q, k, v):
         raise ValueError("q, k, v shapes differ")
 
 
+def _check_tensor(name: str, t: Optional[torch.Tensor], shape, dtype, device) -> None:
+    """A caller-supplied buffer the library writes or reads by pointer: the C
+    side cannot see its size, so dtype, shape, contiguity and device are
+    checked here, before the call (a wrong one would mean out-of-bounds
+    device accesses)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != torch.device(device):
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _check_out(q: torch.Tensor, o: Optional[torch.Tensor], lse: Optional[torch.Tensor],
+               mass: Optional[torch.Tensor] = None) -> None:
+    """o like q (bf16 [N, H, d]), lse float32 [H, N], mass float32 [H, nB, nB]; same device as q."""
+    N, H, _ = q.shape
+    nB = math.ceil(N / 128)
+    _check_tensor("o", o, q.shape, torch.bfloat16, q.device)
+    _check_tensor("lse", lse, (H, N), torch.float32, q.device)
+    _check_tensor("mass", mass, (H, nB, nB), torch.float32, q.device)
+
+
+def _check_workspace(ws: Optional[torch.Tensor], device) -> None:
+    if ws is None:
+        return
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous() or ws.device != torch.device(device):
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+
+
 # ----------------------------------------------------------------- calls ---
 def lvsa_build_index(T: int, T_per: int, W: int, C: int, step: int,
                      frames: Optional[torch.Tensor] = None, counts: Optional[torch.Tensor] = None,
                      device=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor, bool]:
     """A(t) for every frame at ``step``: (frames [T,T] int32, counts [T] int32, over_budget)."""
     dev = device if device is not None else (frames.device if frames is not None else "cuda")
+    _check_tensor("frames", frames, (T, T), torch.int32, dev)
+    _check_tensor("counts", counts, (T,), torch.int32, dev)
     if frames is None:
         frames = torch.empty((T, T), dtype=torch.int32, device=dev)
     if counts is None:
@@ -151,6 +189,8 @@ def lvsa_build_index_window(T: int, T_per: int, W: int, step: int,
                             device=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """A(t) under the fixed-window reading (W non-anchor frames): (frames [T,T] int32, counts [T] int32)."""
     dev = device if device is not None else (frames.device if frames is not None else "cuda")
+    _check_tensor("frames", frames, (T, T), torch.int32, dev)
+    _check_tensor("counts", counts, (T,), torch.int32, dev)
     if frames is None:
         frames = torch.empty((T, T), dtype=torch.int32, device=dev)
     if counts is None:
@@ -161,21 +201,31 @@ def lvsa_build_index_window(T: int, T_per: int, W: int, step: int,
 
 
 def lvsa_index(T: int, frames: torch.Tensor, counts: torch.Tensor) -> bsa_index:
+    """Index of kind BSA_INDEX_LVSA_FRAMES over device frames [T, T] and counts [T] (int32)."""
+    _check_tensor("frames", frames, (T, T), torch.int32, frames.device)
+    _check_tensor("counts", counts, (T,), torch.int32, frames.device)
     ix = bsa_index()
     ix.kind = BSA_INDEX_LVSA_FRAMES
     ix.T = T
     ix.frames = frames.data_ptr()
     ix.counts = counts.data_ptr()
+    ix._tensors = (frames, counts)         # the struct holds raw pointers: keep the tensors alive with it
     return ix
 
 
 def block_index(idx: torch.Tensor, cnt: torch.Tensor, block: int = 128) -> bsa_index:
+    """Index of kind BSA_INDEX_BLOCKS over device idx [H, nQB, nKB] and cnt [H, nQB] (int32)."""
+    if not isinstance(idx, torch.Tensor) or idx.dim() != 3:
+        raise ValueError("idx must be an int32 tensor [H, nQB, nKB]")
     H, nQB, nKB = idx.shape
+    _check_tensor("idx", idx, (H, nQB, nKB), torch.int32, idx.device)
+    _check_tensor("cnt", cnt, (H, nQB), torch.int32, idx.device)
     ix = bsa_index()
     ix.kind = BSA_INDEX_BLOCKS
     ix.block, ix.H, ix.nQB, ix.nKB = block, H, nQB, nKB
     ix.idx = idx.data_ptr()
     ix.cnt = cnt.data_ptr()
+    ix._tensors = (idx, cnt)               # the struct holds raw pointers: keep the tensors alive with it
     return ix
 
 
@@ -187,6 +237,7 @@ def lvsa_block_index(T: int, frames: torch.Tensor, counts: torch.Tensor, idx: to
     ix.T = T
     ix.frames = frames.data_ptr()
     ix.counts = counts.data_ptr()
+    ix._tensors = (frames, counts, idx, cnt)
     return ix
 
 
@@ -203,6 +254,8 @@ def blocksparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, inde
                          stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Masked attention restricted to ``index``; returns (o [N,H,d] bf16, lse [H,N] f32)."""
     _check_qkv(q, k, v)
+    _check_out(q, o, lse)
+    _check_workspace(workspace, q.device)
     N, H, d = q.shape
     if scale is None:
         scale = d ** -0.5
@@ -225,7 +278,10 @@ def blocksparse_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
                                  stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """blocksparse_attn_fwd without a workspace: the library's static scratch array is
     used instead, so the call allocates nothing (o and lse are the caller's)."""
+    if o is None or lse is None:
+        raise ValueError("blocksparse_attn_fwd_noalloc writes into the caller's o and lse")
     _check_qkv(q, k, v)
+    _check_out(q, o, lse)
     N, H, d = q.shape
     if scale is None:
         scale = d ** -0.5
@@ -245,6 +301,8 @@ def attn_dense_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bloc
     When omitted, ``workspace_bytes(BSA_OP_DENSE_BLOCKMASS, ...)`` bytes are allocated.
     """
     _check_qkv(q, k, v)
+    _check_out(q, o, lse, mass)
+    _check_workspace(workspace, q.device)
     N, H, d = q.shape
     nB = math.ceil(N / 128)
     if scale is None:
@@ -259,7 +317,7 @@ def attn_dense_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bloc
         workspace = torch.empty(workspace_bytes(BSA_OP_DENSE_BLOCKMASS, N, H, d), dtype=torch.uint8,
                                 device=q.device)
     rc = _lib.attn_dense_blockmass(_ptr(q), _ptr(k), _ptr(v), N, H, d, block, float(scale),
-                                   _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel(),
+                                   _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _stream(stream))
     _check("attn_dense_blockmass", rc)
     return o, lse, mass
@@ -270,6 +328,8 @@ def attn_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, index: bsa
                    workspace: Optional[torch.Tensor] = None, stream=None):
     """Attention restricted to ``index`` plus its LoSA block mass; returns (o, lse, mass [H, nB, nB] f32)."""
     _check_qkv(q, k, v)
+    _check_out(q, o, lse, mass)
+    _check_workspace(workspace, q.device)
     N, H, d = q.shape
     nB = math.ceil(N / 128)
     if scale is None:
@@ -284,7 +344,7 @@ def attn_blockmass(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, index: bsa
         workspace = torch.empty(workspace_bytes(BSA_OP_BLOCKMASS, N, H, d, index), dtype=torch.uint8,
                                 device=q.device)
     rc = _lib.attn_blockmass(_ptr(q), _ptr(k), _ptr(v), N, H, d, float(scale), ctypes.byref(index),
-                             _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel(), _stream(stream))
+                             _ptr(o), _ptr(lse), _ptr(mass), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check("attn_blockmass", rc)
     return o, lse, mass
 
@@ -294,6 +354,8 @@ def losa_select(mass: torch.Tensor, tau: float = 0.99, idx=None, cnt=None, strea
     if mass.dtype != torch.float32 or not mass.is_cuda or not mass.is_contiguous() or mass.dim() != 3:
         raise ValueError("mass must be a contiguous float32 CUDA tensor [H, nQB, nKB]")
     H, nQB, nKB = mass.shape
+    _check_tensor("idx", idx, (H, nQB, nKB), torch.int32, mass.device)
+    _check_tensor("cnt", cnt, (H, nQB), torch.int32, mass.device)
     if idx is None:
         idx = torch.empty((H, nQB, nKB), dtype=torch.int32, device=mass.device)
     if cnt is None:

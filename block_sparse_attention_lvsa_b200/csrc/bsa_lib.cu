@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "ptx.cuh"
@@ -74,14 +75,15 @@ template <int D, bool MASS>
 int launch_attn(const void* q, const void* k, const void* v, int N, int H, int grid_heads, const AttnParams& prm,
                 cudaStream_t st) {
   using L = AttnSmem<D, MASS>;
-  static bool attr_set[kMaxDevices] = {};
+  // set once per device; concurrent first calls may both set it (idempotent)
+  static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(attn_tile_kernel<D, MASS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(L::kAlloc)) != cudaSuccess)
       return BSA_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   CUtensorMap mq, mk, mv;
   // query, key and value tiles are all 128 rows (boxes of 128 rows x 64 channels)
@@ -364,15 +366,15 @@ int losa_select(const float* mass, int H, int nQB, int nKB, double tau, int32_t*
   const size_t row_bytes = static_cast<size_t>(nKB) * 8;
   const int wpc = static_cast<int>(std::min<size_t>(8, std::max<size_t>(1, (96 * 1024) / row_bytes)));
   const size_t smem = row_bytes * wpc;
-  static bool attr_set[kMaxDevices] = {};
+  static std::atomic<bool> attr_set[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_acquire)) {
     // largest request: 96 KB (several warps) or one row of kSelectMaxBlocks keys (64 KB)
     if (cudaFuncSetAttribute(losa_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
         cudaSuccess)
       return BSA_ERR_CUDA;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const long long ctas = std::min<long long>((rows + wpc - 1) / wpc, 1LL << 20);
   losa_select_kernel<<<static_cast<unsigned>(ctas), wpc * 32, smem, st>>>(mass, static_cast<int>(rows), nKB, tau,
@@ -432,11 +434,12 @@ std::mutex g_noalloc_mu;
 extern "C" int blocksparse_attn_fwd_noalloc(const void* q, const void* k, const void* v, int N, int H, int d,
                                             float scale, const bsa_index* index, void* o, float* lse,
                                             void* stream) {
-  if (!index || N < 1) return BSA_ERR_ARG;
-  if (index->kind == BSA_INDEX_LVSA_FRAMES) {
+  if (!index || N < 1 || H < 1) return BSA_ERR_ARG;
+  if (index->kind == BSA_INDEX_LVSA_FRAMES || index->kind == BSA_INDEX_LVSA_BLOCKS) {
+    // frame lists need the tile lists; the intersection also H * nB * nB flag bytes
     if (index->T < 1 || index->T > kMaxFrames) return BSA_ERR_ARG;
     if (N % index->T) return BSA_ERR_SHAPE;
-    if (lvsa_ws_layout(N, index->T).total > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;
+    if (index_ws_bytes(index, N, H) > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;
   }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BSA_ERR_CUDA;

@@ -273,12 +273,16 @@ int blocksparse_attn_fwd(const void* q, const void* k, const void* v,
  * lists) lives in one file-scope device array of BSA_NOALLOC_SCRATCH_BYTES
  * bytes that every GPU loading the library holds until the process exits.
  *
- * Arguments, layouts and results are those of blocksparse_attn_fwd (both
- * index kinds are accepted; block indexes need no scratch).  Returns
- * BSA_ERR_WORKSPACE, before anything is enqueued, when an LVSA frame index
- * needs more scratch than BSA_NOALLOC_SCRATCH_BYTES, i.e. when
- * bsa_workspace_bytes(BSA_OP_BLOCKSPARSE_FWD, ...) exceeds it (up to about
- * N = 234,000 tokens fits).
+ * Arguments, layouts and results are those of blocksparse_attn_fwd, and all
+ * three index kinds are accepted.  Block indexes (BSA_INDEX_BLOCKS) need no
+ * scratch.  LVSA frame indexes (BSA_INDEX_LVSA_FRAMES) need the frame-pair
+ * bit matrix and the key-tile lists, about 5 * ceil(N/128)^2 bytes: up to
+ * about N = 234,000 tokens fits.  The intersection (BSA_INDEX_LVSA_BLOCKS)
+ * needs H * ceil(N/128)^2 bytes more for its per-head flags, so it fits only
+ * small shapes (N = 32,760 with up to 250 heads; not the 14B-head 720p shape).
+ * The need is bsa_workspace_bytes(BSA_OP_BLOCKSPARSE_FWD, ...); when it is
+ * larger than BSA_NOALLOC_SCRATCH_BYTES the call returns BSA_ERR_WORKSPACE
+ * before anything is enqueued.
  *
  * The first call on a device looks up the device address of the array on
  * that device (cudaGetSymbolAddress, with that device current); make that

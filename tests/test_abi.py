@@ -141,3 +141,37 @@ def test_host_validation_rejects_before_launch(bsa):
     assert s(fake, 2, 4, 9000, 0.99, fake, fake, nul) == bsa.BSA_ERR_UNSUPPORTED
     assert L.bsa_debug_expired_wait(10, 0, nul) == bsa.BSA_ERR_ARG
     assert L.bsa_debug_expired_wait(1_000_000, 2, nul) == bsa.BSA_ERR_ARG
+
+
+def test_output_checks_reject_wrong_buffers(bsa):
+    """Caller-supplied outputs and index arrays are checked before any call:
+    the library sees only pointers, so an undersized or mistyped buffer would
+    mean out-of-bounds device writes (CPU tensors stand in for device ones)."""
+    import torch
+    N, H, d = 300, 2, 64
+    q = torch.zeros((N, H, d), dtype=torch.bfloat16)
+    ok_o = torch.zeros_like(q)
+    ok_lse = torch.zeros((H, N), dtype=torch.float32)
+    bsa._check_out(q, ok_o, ok_lse)                                     # accepted
+    bad = [
+        (torch.zeros((N, H, d), dtype=torch.float32), ok_lse),          # o dtype
+        (torch.zeros((N - 1, H, d), dtype=torch.bfloat16), ok_lse),     # o shape
+        (torch.zeros((N, H, 2 * d), dtype=torch.bfloat16)[:, :, ::2], ok_lse),   # o not contiguous
+        (ok_o, torch.zeros((N, H), dtype=torch.float32)),               # lse transposed
+        (ok_o, torch.zeros((H, N), dtype=torch.float64)),               # lse dtype
+        (ok_o.to("meta"), ok_lse),                                      # o on another device
+    ]
+    for o, lse in bad:
+        with pytest.raises(ValueError):
+            bsa._check_out(q, o, lse)
+    nB = 3
+    with pytest.raises(ValueError):
+        bsa._check_out(q, ok_o, ok_lse, torch.zeros((H, nB, nB - 1), dtype=torch.float32))
+    with pytest.raises(ValueError):                                     # int64 block index
+        bsa.block_index(torch.zeros((H, nB, nB), dtype=torch.int64), torch.zeros((H, nB), dtype=torch.int32))
+    with pytest.raises(ValueError):                                     # cnt of the wrong shape
+        bsa.block_index(torch.zeros((H, nB, nB), dtype=torch.int32), torch.zeros((H, nB + 1), dtype=torch.int32))
+    with pytest.raises(ValueError):                                     # frames not [T, T]
+        bsa.lvsa_index(5, torch.zeros((5, 4), dtype=torch.int32), torch.zeros(5, dtype=torch.int32))
+    with pytest.raises(ValueError):                                     # no-alloc needs o and lse
+        bsa.blocksparse_attn_fwd_noalloc(q, q, q, bsa.bsa_index(), None, None)
