@@ -349,7 +349,8 @@ __device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, floa
 template <int D, bool MASS>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                 const AttnParams p) {
   using L = AttnSmem<D, MASS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -670,14 +671,26 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (bad && r == 0) set_status(BSA_ERR_INDEX_RANGE);
 
     {
-      // ---- epilogue: O / l (bf16) and LSE for this group's query tile
+      // ---- epilogue: O / l (bf16) and LSE for this group's query tile.  The
+      // group's Q tile in shared memory is idle now (its last QK^T completed
+      // before its last PV, which PVDONE covers; with no tile at all, once its
+      // load has landed): each thread writes its
+      // row of O there in the 128-byte-swizzled layout of the TMA box (16-byte
+      // chunk c of row r at chunk position c ^ (r & 7), so the eight rows of
+      // every quarter warp hit distinct banks), and one thread stores the
+      // whole tile with TMA (rows past N are clipped by the tensor map):
+      // global writes are whole 128-byte rows instead of 16 bytes in each of
+      // 32 rows per warp store.
       if (ok && cnt > 0) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_PVDONE + x), (cnt - 1) & 1, limit));
         tc_fence_after();
       }
       const bool have = __all_sync(0xFFFFFFFFu, ok && cnt > 0);
+      // a group that processed no tile (empty list) may get here before the
+      // TMA load of its Q tile has landed: wait for it before reusing the buffer
+      if (cnt == 0 && any_work) __all_sync(0xFFFFFFFFu, mbar_wait(bar(B_QFULL), 0, limit));
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(q) * p.H + h) * D;
+      const uint32_t sO = base + L::kQ + x * L::kTile;
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t ov[32];
@@ -688,18 +701,24 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
           for (int c = 0; c < 32; ++c) ov[c] = 0u;
         }
-        if (q < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv, __uint_as_float(ov[8 * v4 + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv, __uint_as_float(ov[8 * v4 + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv, __uint_as_float(ov[8 * v4 + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv);
-            dst[v4] = w;
-          }
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const int col = c0 + 8 * v4;                  // first of 8 channels in this 16-byte chunk
+          const uint32_t dst = sO + (col / 64) * L::kBox + r * 128 + ((((col % 64) / 8) ^ (r & 7)) * 16);
+          st_shared_v4(dst,
+                       pack_bf16x2(__uint_as_float(ov[8 * v4 + 0]) * inv, __uint_as_float(ov[8 * v4 + 1]) * inv),
+                       pack_bf16x2(__uint_as_float(ov[8 * v4 + 2]) * inv, __uint_as_float(ov[8 * v4 + 3]) * inv),
+                       pack_bf16x2(__uint_as_float(ov[8 * v4 + 4]) * inv, __uint_as_float(ov[8 * v4 + 5]) * inv),
+                       pack_bf16x2(__uint_as_float(ov[8 * v4 + 6]) * inv, __uint_as_float(ov[8 * v4 + 7]) * inv));
         }
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(1 + x, 128);                   // the group's 128 rows are in shared memory
+      if (r == 0 && qt < p.nB) {
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b) tma_store_3d(&tmO, sO + b * L::kBox, b * 64, h, qt * 128);
+        bulk_commit();
+        bulk_wait_read_all();                           // shared memory read before the CTA may exit
       }
       if (q < p.N) {
         p.lse[static_cast<size_t>(h) * p.N + q] =

@@ -85,13 +85,13 @@ int launch_attn(const void* q, const void* k, const void* v, int N, int H, int g
       return BSA_ERR_CUDA;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  CUtensorMap mq, mk, mv;
-  // query, key and value tiles are all 128 rows (boxes of 128 rows x 64 channels)
+  CUtensorMap mq, mk, mv, mo;
+  // query, key, value and output tiles are all 128 rows (boxes of 128 rows x 64 channels)
   if (!make_qkv_map(&mq, q, N, H, D, 128) || !make_qkv_map(&mk, k, N, H, D, 128) ||
-      !make_qkv_map(&mv, v, N, H, D, 128))
+      !make_qkv_map(&mv, v, N, H, D, 128) || !make_qkv_map(&mo, prm.o, N, H, D, 128))
     return BSA_ERR_CUDA;
   dim3 grid((prm.nB + kQTilesPerCta - 1) / kQTilesPerCta, grid_heads);
-  attn_tile_kernel<D, MASS><<<grid, kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, prm);
+  attn_tile_kernel<D, MASS><<<grid, kAttnThreads, L::kAlloc, st>>>(mq, mk, mv, mo, prm);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }
 
