@@ -135,10 +135,8 @@ int blockmass_passes(const void* q, const void* k, const void* v, int N, int H, 
     p.h_off = h0;
     int rc = launch_attn_any(d, true, q, k, v, N, H, hn, p, st);
     if (rc != BSA_OK) return rc;
-    const long long warps = static_cast<long long>(hn) * nB * nB;
-    const long long blocks = (warps + kMassThreads / 32 - 1) / (kMassThreads / 32);
-    if (blocks > 0x7FFFFFFFLL) return BSA_ERR_UNSUPPORTED;
-    blockmass_reduce_kernel<<<static_cast<unsigned>(blocks), kMassThreads, 0, st>>>(lpart, lse, mass, N, nB, h0, hn);
+    const dim3 grid((nB + kMassWarps - 1) / kMassWarps, (nB + kMassKt - 1) / kMassKt, hn);
+    blockmass_reduce_kernel<<<grid, kMassThreads, 0, st>>>(lpart, lse, mass, N, nB, h0);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   return BSA_OK;
