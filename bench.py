@@ -9,21 +9,29 @@ generated before timing; every tensor is 604 MB, larger than L2, so no flush
 is needed between steps).  The metric counts FLOPs on kept 128x128 tiles
 (4 * d * 128 * 128 per tile and head).
 
-Also measured in the same run (reported as extra keys): the same kernel run
-dense (every tile), the exact-pair FLOP rate, and the LoSA path on the
-14B-shaped workload (dense measuring step with block mass, 99% selection,
-frozen-index sparse steps).
+Every other workload is measured in the same run at its full size and
+reported as an extra key (`configs`): the tiny case, the 1x-horizon shapes
+(C = 21 equal to dense, and C = 11), the balanced 6x variant, the LoSA path
+on the 14B-shaped workload (dense measuring step with block mass, 99%
+selection, the 39 frozen-index steps on their own perturbed inputs), the
+720p 14B-head shape at all 40 heads (LVSA, LoSA alone, LoSA inside LVSA) and
+the HunyuanVideo-1.5-shaped horizons with the attention path's peak memory.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {b200,reference}]
-Multi-GPU: launched by torchrun; each rank runs its own replica of the
-workload (independent problems, no data-path collective): weak scaling.
+Multi-GPU: one process per GPU.  Under torchrun (WORLD_SIZE set) --gpus must
+equal the world size; without a launcher and N > 1, bench.py starts the N
+ranks itself through torch.distributed.run.  Each rank runs its own replica
+of the workload (independent problems, no data-path collective): weak
+scaling; --shard heads splits one problem by heads instead (strong scaling).
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -42,6 +50,7 @@ METRIC = "effective TFLOP/s (kept blocks) & ms/call, Wan-1.3B shape 6x horizon; 
 UNIT = "TFLOP/s"
 WORKLOAD = "wan1.3b_6x"
 POOL = 3            # distinct fresh input sets cycled through the steps
+LVSA_WORKLOADS = [n for n, w in WORKLOADS.items() if w.C is not None]
 
 
 def load_peaks():
@@ -55,10 +64,30 @@ def load_peaks():
 
 
 # ------------------------------------------------------------ distributed --
+def free_port() -> int:
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def launch_ranks(n: int, argv) -> int:
+    """Start `n` ranks of this script through torch.distributed.run (one
+    process per GPU, rendezvous on 127.0.0.1) and return their exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
 def dist_init(n_gpus):
+    """Join the process group when launched as one of several ranks; the
+    world size must equal --gpus."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch one rank per GPU")
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -77,24 +106,24 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _reduce(x: float, world: int, op) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    import torch.distributed as dist
+    return _reduce(x, world, dist.ReduceOp.MAX if world > 1 else None)
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
     import torch.distributed as dist
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(x, world, dist.ReduceOp.SUM if world > 1 else None)
 
 
 # ----------------------------------------------------------------- clocks --
@@ -118,6 +147,10 @@ class ClockSampler:
                  "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+        # nvidia-smi takes a moment to start: wait (up to 5 s) for its first sample
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 5.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.05)
         return self
 
     def __exit__(self, *a):
@@ -156,75 +189,155 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------- CPU baseline --
-def oracle_sample(wl, step, rows_n, head, qkv=None, seed=0):
-    """Time the oracle on a bounded sample: ``rows_n`` query rows of one head.
+CPU_ROWS_PER_HEAD = 24576     # stratified query rows per sampled head
+CPU_HEADS = 2                 # heads per sample
 
-    Returns (seconds, kept-tile-equivalent FLOPs of the sample, rows, cores).
-    The kept-tile-equivalent FLOPs are the workload's kept-tile FLOPs per
-    head-row times the number of sampled rows, so the rate is in the same
-    accounting as the GPU metric.
+
+def oracle_sample(pool, wl, step, rows_per_head, heads, seed, qkv=None):
+    """Time the oracle, spread over the host cores, on a bounded sample of
+    one LVSA step: `rows_per_head` stratified query rows of each of `heads`.
+
+    Returns (seconds of the parallel oracle evaluation, kept-tile-equivalent
+    FLOPs of the sample, rows).  The kept-tile-equivalent FLOPs of a row are
+    the workload's kept-tile FLOPs per head-row of its query tile, so the
+    rate is in the accounting of the GPU metric.
     """
-    import numpy as np
-    from oracle import attention as oatt
     from oracle import lvsa as olvsa
     from oracle import tiles as otiles
     if qkv is None:
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         qkv = inputs.workload_qkv(wl, step, device=dev)
-    q, k, v = (x[:, head:head + 1, :].to("cpu").to(torch.float64).numpy() for x in qkv)
     A, _ = olvsa.attended_frames(wl.T, wl.T_per, wl.W, wl.C, step)
-    rows = inputs.sample_rows(wl.N, wl.P, rows_n, seed).numpy()
-    t0 = time.perf_counter()
-    oatt.attention_rows(q, k, v, wl.scale, rows, [0],
-                        lambda h, r: olvsa.allowed_keys_for_row(r, A, wl.P, wl.N),
-                        lambda h, r: r // wl.P)
-    dt = time.perf_counter() - t0
-    idx, _ = otiles.kept_tiles(A, wl.T, wl.N, qtiles=sorted(set((rows // 128).tolist())))
-    per_qtile = {qt: len(r) for qt, r in zip(sorted(set((rows // 128).tolist())), idx)}
-    flops = sum(4 * wl.d * 128 * per_qtile[r // 128] for r in rows)   # kept-tile FLOPs per row
-    cores = len(os.sched_getaffinity(0))
-    return dt, flops, len(rows), cores
+    rows = inputs.sample_rows(wl.N, wl.P, rows_per_head, seed).numpy()
+    work = []
+    for h in heads:
+        q, k, v = (x[:, h:h + 1, :].to("cpu").to(torch.float64).numpy() for x in qkv)
+        work.append((pool.put_head(q, k, v), rows))
+    _, dt = pool.attention_rows(work, lambda r: olvsa.allowed_keys_for_row(r, A, wl.P, wl.N),
+                                lambda r: r // wl.P, wl.scale)
+    pool.drop_files()
+    qts = sorted(set((rows // 128).tolist()))
+    idx, _ = otiles.kept_tiles(A, wl.T, wl.N, qtiles=qts)
+    per_qtile = {qt: len(r) for qt, r in zip(qts, idx)}
+    flops = len(heads) * sum(4 * wl.d * 128 * per_qtile[r // 128] for r in rows.tolist())
+    return dt, flops, len(rows) * len(heads)
+
+
+def sample_note(pool, wl):
+    return (f"{CPU_HEADS} heads x {CPU_ROWS_PER_HEAD} stratified query rows (frame and tile boundaries, last "
+            f"partial tile) of one LVSA step of {wl.name}, fp64 numpy oracle, {pool.workers} single-threaded "
+            "worker processes over (head, query frame) tasks; kept-tile-equivalent FLOPs")
 
 
 def run_reference(args, rank, world):
-    """Oracle arm: the fp64 CPU oracle timed on this host's cores."""
+    """Oracle arm: the fp64 CPU oracle timed on this host's cores, on a bounded
+    sample of the workload per step (rank 0 only)."""
     if rank != 0:
         return
-    wl = WORKLOADS[WORKLOAD]
-    rows_n = 48
+    from oracle.pool import OraclePool
+    wl = WORKLOADS[args.workload]
+    pool = OraclePool()
     dev = "cuda" if torch.cuda.is_available() else "cpu"
+    rows_n = min(CPU_ROWS_PER_HEAD, wl.N)
+    heads = list(range(min(CPU_HEADS, wl.H)))
     secs, flops = [], []
-    cores = len(os.sched_getaffinity(0))
-    for i in range(args.warmup + args.steps):
-        s = i % wl.steps
-        qkv = inputs.workload_qkv(wl, s, device=dev)
-        dt, fl, n, cores = oracle_sample(wl, s, rows_n, head=s % wl.H, qkv=qkv, seed=100 + i)
-        del qkv
-        if i >= args.warmup:
-            secs.append(dt)
-            flops.append(fl)
+    try:
+        for i in range(args.warmup + args.steps):
+            s = i % wl.steps
+            qkv = inputs.workload_qkv(wl, s, device=dev)
+            dt, fl, n = oracle_sample(pool, wl, s, rows_n, [(h + s) % wl.H for h in heads], 100 + i, qkv)
+            del qkv
+            if i >= args.warmup:
+                secs.append(dt)
+                flops.append(fl)
+    finally:
+        workers = pool.workers
+        note = sample_note(pool, wl)
+        pool.close()
     value = sum(flops) / sum(secs) / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000 * sum(secs) / len(secs), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block(wl, world),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{rows_n} query rows of one head per step (stratified), fp64 numpy, "
-                                       "value in kept-tile-equivalent FLOPs"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": note},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def config_block(wl, world, shard="replicas", H_total=None):
     H_all = wl.H if H_total is None else H_total
-    return {"workload": f"{wl.name}: LVSA block-sparse self-attention, Wan-2.1-1.3B shape at 6x horizon, "
-                        f"T={wl.T} frames x P={wl.P} tokens (N={wl.N}), H={H_all}, d={wl.d}, "
-                        f"C={wl.C}, W={wl.W}, T_per={wl.T_per}, anchors rotated per step, fresh q/k/v per step",
+    return {"workload": f"{wl.name}: LVSA block-sparse self-attention, T={wl.T} frames x P={wl.P} tokens "
+                        f"(N={wl.N}), H={H_all}, d={wl.d}, C={wl.C}, W={wl.W}, T_per={wl.T_per}, anchors "
+                        "rotated per step, fresh q/k/v per step",
             "N": wl.N, "H": H_all, "d": wl.d, "T": wl.T, "P": wl.P, "C": wl.C, "W": wl.W, "T_per": wl.T_per,
             "global_batch": world if shard == "replicas" else 1, "seq_len": wl.N,
             "parallelism": f"{shard} x{world}",
-            "l2": "inputs larger than L2 (604 MB per tensor), no flush"}
+            "l2": "inputs larger than L2 (604 MB per tensor), no flush" if wl.N * wl.H * wl.d * 2 > 126e6
+                  else "inputs smaller than L2"}
+
+
+# ---------------------------------------------------------------- helpers --
+def ev_timed(fn, reps, stream, warm=1):
+    """Median ms of `fn` between CUDA events on `stream` over `reps` calls
+    (after `warm` untimed calls)."""
+    out = []
+    for i in range(warm + reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= warm:
+            out.append(a.elapsed_time(b))
+    return statistics.median(out)
+
+
+def graph_timed(fn, n, reps=5):
+    """Median ms per call of `fn` captured `n` times into one CUDA graph (so the
+    host-side cost of each call is not part of the measurement)."""
+    fn()                                   # first call on the device does its set-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(n):
+                fn()
+    out = []
+    for i in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        if i:
+            out.append(a.elapsed_time(b) / n)
+    del g
+    return statistics.median(out)
+
+
+def rates(flop_kept, flop_exact, ms, peaks):
+    """TFLOP/s on kept tiles and exact pairs, and fractions of the burst peak."""
+    tk = flop_kept / (ms / 1e3) / 1e12
+    te = flop_exact / (ms / 1e3) / 1e12
+    return {"ms_per_call": ms, "tflops_kept_tiles": tk, "tflops_exact_pairs": te,
+            "frac_of_bf16_burst": tk / peaks["bf16"], "frac_exact_of_bf16_burst": te / peaks["bf16"]}
+
+
+def lvsa_tiles(bsa, wl, s, frames, counts, ws, qkv, o, lse):
+    """Kept 128x128 tiles (per head) and exact allowed pairs of step s, from
+    the library's own tile lists."""
+    bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, s, frames, counts)
+    ix = bsa.lvsa_index(wl.T, frames, counts)
+    bsa.blocksparse_attn_fwd(*qkv, ix, scale=wl.scale, o=o, lse=lse, workspace=ws)
+    _, tcnt, _, _ = bsa.lvsa_workspace_views(ws, wl.N, wl.T)
+    return int(tcnt.sum().item()), int(counts.sum().item()) * wl.P * wl.P
+
+
+def dense_frames(T, dev):
+    f = torch.arange(T, dtype=torch.int32, device=dev).repeat(T, 1).contiguous()
+    return f, torch.full((T,), T, dtype=torch.int32, device=dev)
 
 
 # ------------------------------------------------------------------ main --
@@ -233,51 +346,49 @@ def run_b200(args, rank, world, local):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU (the product path has no CPU fallback)")
     peaks = load_peaks()
-    wl = WORKLOADS[WORKLOAD]
+    wl = WORKLOADS[args.workload]
     if args.heads:
-        import dataclasses
         wl = dataclasses.replace(wl, H=args.heads)      # profiling case only
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
-    N, H, d = wl.N, wl.H, wl.d
-    nB = math.ceil(N / 128)
+
+    # the CPU-baseline pool starts (spawn) before any GPU work of this process
+    pool = None
+    if rank == 0 and not args.no_cpu_baseline and not args.main_only:
+        from oracle.pool import OraclePool
+        pool = OraclePool()
 
     # ---- inputs (fresh per step, cycled from a pool), outputs, index buffers
     H_total = wl.H
     if args.shard == "heads":
         # one problem split by heads: every rank draws the same inputs and keeps its head range
         from block_sparse_attention_lvsa_b200 import heads
-        import dataclasses
         h0, h1 = heads.head_range(wl.H, world, rank)
         if h1 == h0:
             raise SystemExit("--shard heads needs at least as many heads as ranks")
-        pool = [tuple(heads.local_heads(x, wl.H, world, rank) for x in inputs.workload_qkv(wl, s, device=dev))
-                for s in range(POOL)]
+        qpool = [tuple(heads.local_heads(x, wl.H, world, rank) for x in inputs.workload_qkv(wl, s, device=dev))
+                 for s in range(POOL)]
         wl = dataclasses.replace(wl, H=h1 - h0)
-        H = wl.H
     else:
-        pool = [inputs.workload_qkv(inputs_wl(wl, rank), s, device=dev) for s in range(POOL)]
-    o = torch.empty_like(pool[0][0])
+        qpool = [inputs.workload_qkv(inputs_wl(wl, rank), s, device=dev) for s in range(POOL)]
+    N, H, d = wl.N, wl.H, wl.d
+    nB = math.ceil(N / 128)
+    o = torch.empty_like(qpool[0][0])
     lse = torch.empty((H, N), dtype=torch.float32, device=dev)
     frames = torch.empty((wl.T, wl.T), dtype=torch.int32, device=dev)
     counts = torch.empty((wl.T,), dtype=torch.int32, device=dev)
     ix = bsa.lvsa_index(wl.T, frames, counts)
-    ws_bytes = bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix), dtype=torch.uint8, device=dev)
 
     # kept tiles and exact pairs per anchor phase (s mod T_per), from the library's own lists
     kept_tiles, exact_pairs = {}, {}
     for ph in range(wl.T_per):
-        bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, ph, frames, counts)
-        bsa.blocksparse_attn_fwd(*pool[0], ix, scale=wl.scale, o=o, lse=lse, workspace=ws)
-        _, tcnt, _, _ = bsa.lvsa_workspace_views(ws, N, wl.T)
-        kept_tiles[ph] = int(tcnt.sum().item())
-        exact_pairs[ph] = int(counts.sum().item()) * wl.P * wl.P
+        kept_tiles[ph], exact_pairs[ph] = lvsa_tiles(bsa, wl, ph, frames, counts, ws, qpool[0], o, lse)
     assert bsa.get_device_status() == bsa.BSA_OK
 
     def step(i, ev=None):
         s = i % wl.steps
-        q, k, v = pool[i % POOL]
+        q, k, v = qpool[i % POOL]
         bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, s, frames, counts, stream=stream)
         if ev is not None:
             ev[0].record(stream)
@@ -286,16 +397,15 @@ def run_b200(args, rank, world, local):
             ev[1].record(stream)
         return s
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     phases = []
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk:            # sampling covers the warm-up and the timed steps
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
         t_start.record(stream)
         for i in range(args.steps):
             phases.append(step(args.warmup + i, evs[i]) % wl.T_per)
@@ -314,6 +424,7 @@ def run_b200(args, rank, world, local):
     job_flop = sum_over_ranks(float(sum(flop_tile)), world)
     value = job_flop / (max_total_ms / 1e3) / 1e12
     achieved = sum(flop_tile) / (sum(call_ms) / 1e3) / 1e12          # per-launch, this rank
+    achieved_exact = sum(flop_exact) / (sum(call_ms) / 1e3) / 1e12
     clocks = clk.summary()
 
     if args.main_only:
@@ -323,35 +434,23 @@ def run_b200(args, rank, world, local):
         return
 
     # ---- dense run of the same kernel (every tile kept), same inputs
-    dframes = torch.arange(wl.T, dtype=torch.int32, device=dev).repeat(wl.T, 1).contiguous()
-    dcounts = torch.full((wl.T,), wl.T, dtype=torch.int32, device=dev)
+    dframes, dcounts = dense_frames(wl.T, dev)
     dix = bsa.lvsa_index(wl.T, dframes, dcounts)
-    dense_ms = []
-    for i in range(3):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        bsa.blocksparse_attn_fwd(*pool[i % POOL], dix, scale=wl.scale, o=o, lse=lse, workspace=ws, stream=stream)
-        b.record(stream)
-        torch.cuda.synchronize()
-        if i > 0:
-            dense_ms.append(a.elapsed_time(b))
-    dense_ms = statistics.median(dense_ms)
+    dense_ms = ev_timed(lambda: bsa.blocksparse_attn_fwd(*qpool[1], dix, scale=wl.scale, o=o, lse=lse, workspace=ws,
+                                                         stream=stream), 2, stream)
     dense_flop = 4 * d * H * nB * nB * 128 * 128
-    sdpa = run_sdpa_context(pool[0], wl.scale, stream) if rank == 0 else None
+    sdpa = run_sdpa_context(qpool[0], wl.scale, stream) if rank == 0 else None
     index_us = graph_timed(lambda: bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, 1, frames, counts), 50) * 1e3
-
-    # ---- balanced variant of the same shape (T_per = 21: |A(t)| = C = 21 for every t and s)
-    balanced = run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws) if rank == 0 else None
     gather = run_gather(o, lse, H_total, world) if args.shard == "heads" and world > 1 else None
 
     # ---- e2e: host buffers through the public API, copies inside the timed region,
     # over one whole denoising run of the workload (its 40 steps)
-    e2e = run_e2e(bsa, wl, pool[0], stream, frames, counts, ix, o, lse, ws, wl.steps, kept_tiles, world)
-    del pool
+    e2e = run_e2e(bsa, wl, qpool[0], stream, frames, counts, ix, o, lse, ws, wl.steps, kept_tiles, world)
+    del qpool, o, lse, ws
+    torch.cuda.empty_cache()
 
-    # ---- LoSA path on the 14B-shaped workload, and LoSA inside LVSA at 720p (secondary)
-    losa = run_losa(bsa, rank, stream, peaks) if rank == 0 else None
-    lvsa_losa = run_lvsa_losa(bsa, stream) if rank == 0 else None
+    # ---- every other workload at full size (rank 0; replicas would only repeat it)
+    configs = run_configs(bsa, stream, peaks) if rank == 0 and not args.no_configs else None
 
     med_call = statistics.median(call_ms)
     line = {
@@ -361,45 +460,49 @@ def run_b200(args, rank, world, local):
         "data": "synthetic", "config": config_block(wl, world, args.shard, H_total),
         "ms_per_call": med_call,
         "tflops_kept_tiles": achieved,
-        "tflops_exact_pairs": sum(flop_exact) / (sum(call_ms) / 1e3) / 1e12,
+        "tflops_exact_pairs": achieved_exact,
         "frac_of_bf16_burst": achieved / peaks["bf16"],
         "speedup_vs_dense": dense_ms / med_call,
         "dense_ms_per_call": dense_ms,
         "dense_tflops": dense_flop / (dense_ms / 1e3) / 1e12,
         "kept_tile_fraction": statistics.mean(kept_tiles[ph] for ph in phases) / (nB * nB),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_sustained"], "traffic": TRAFFIC_PER_LAUNCH,
-                     "peak_kind": f"bf16 dense, sustained ({peaks['src']}); kernel timed inside back-to-back steps",
-                     "kernel": "attn_tile_kernel<128,false> (+2 index-expansion launches of a few us in the same call)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16"], "traffic": TRAFFIC_PER_LAUNCH,
+                     "frac_exact_pairs": achieved_exact / peaks["bf16"],
+                     "frac_of_sustained_peak": achieved / peaks["bf16_sustained"],
+                     "peak_kind": f"bf16 dense, burst ({peaks['src']}): each ~40 ms call is timed on its own "
+                                  "with CUDA events",
+                     "kernel": "attn_tile_kernel<128,false> (+2 index-expansion launches of a few us in the "
+                               "same call)"},
         "e2e": e2e,
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
-        "losa": losa,
-        "balanced_tper21": balanced,
-        "losa_within_lvsa_720p": lvsa_losa,
         "lvsa_build_index": {"us": index_us, "bytes_out": (wl.T * wl.T + wl.T) * 4,
                              "note": "a few KB written: latency-bound, GB/s not meaningful"},
         "context_torch_sdpa_dense": sdpa,
+        "configs": configs,
     }
     if gather is not None:
         line["gather_heads"] = gather
-    if rank == 0 and not args.no_cpu_baseline:
-        dt, fl, n, cores = oracle_sample(wl, 0, args.cpu_rows, head=0, qkv=None, seed=7)
-        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                "sample": f"{n} stratified query rows of head 0 at step 0 ({dt:.1f} s), fp64 numpy; "
-                                          "kept-tile-equivalent FLOPs",
-                                "rows_per_s": n / dt,
-                                "extrapolated_full_call_s": dt * wl.N * H_total / n}
+    if pool is not None:
+        try:
+            dt, fl, n = oracle_sample(pool, wl, 0, min(CPU_ROWS_PER_HEAD, wl.N), list(range(min(CPU_HEADS, wl.H))),
+                                      seed=7)
+            line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": pool.workers, "kind": "oracle",
+                                    "sample": sample_note(pool, wl) + f" ({dt:.1f} s)",
+                                    "rows_per_s": n / dt,
+                                    "extrapolated_full_call_s": dt * wl.N * H_total / n}
+        finally:
+            pool.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
 # DRAM bytes (read + write) per launch of the attention kernel at the full
-# 12-head workload: the ncu capture of the 4-head case of the same workload
-# (658.5 MB read + 190.7 MB written, step-0 index) scaled by 12/4 - traffic
-# grows with the number of heads.  Must be re-measured (or set to None)
-# whenever the kernel changes.
-TRAFFIC_PER_LAUNCH = 2.548e9
+# 12-head workload, from an ncu capture of the 4-head case of the same
+# workload scaled by 12/4 (traffic grows with the number of heads); None
+# until the counters are taken on the current kernel.
+TRAFFIC_PER_LAUNCH = None
 
 
 def run_gather(o, lse, H, world, reps=3):
@@ -427,105 +530,15 @@ def run_sdpa_context(qkv, scale, stream, reps=2):
     import torch.nn.functional as F
     q, k, v = (x.transpose(0, 1).unsqueeze(0) for x in qkv)       # [1, H, N, d] views
     try:
-        ms = []
-        for i in range(reps + 1):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            out = F.scaled_dot_product_attention(q, k, v, scale=scale)
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i:
-                ms.append(a.elapsed_time(b))
-        del out
+        ms = ev_timed(lambda: F.scaled_dot_product_attention(q, k, v, scale=scale), reps, stream)
         N, H, d = qkv[0].shape
-        return {"ms": statistics.median(ms), "tflops": 4 * d * H * N * N / (statistics.median(ms) / 1e3) / 1e12}
+        return {"ms": ms, "tflops": 4 * d * H * N * N / (ms / 1e3) / 1e12}
     except Exception as e:                                        # noqa: BLE001 - context only
         return {"unavailable": str(e).splitlines()[0][:200]}
 
 
-def run_lvsa_losa(bsa, stream, heads=4):
-    """LoSA's selection inside LVSA's frame sets on the 720p Wan-14B shape
-    (T=63 x P=3600, d=128), `heads` of its 40 heads: the restricted measuring
-    step (LVSA attention + block mass), the selection, and a later step on
-    the intersection index against LVSA alone.  Times scale with heads."""
-    import dataclasses
-    wl = dataclasses.replace(WORKLOADS["720p_14b"], H=heads)
-    N, H, d, nB = wl.N, wl.H, wl.d, math.ceil(wl.N / 128)
-    q, k, v = inputs.workload_qkv(wl, 0, device="cuda")
-    frames, counts, _ = bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, 0, device="cuda")
-    ix = bsa.lvsa_index(wl.T, frames, counts)
-    o = torch.empty_like(q)
-    lse = torch.empty((H, N), dtype=torch.float32, device="cuda")
-    mass = torch.empty((H, nB, nB), dtype=torch.float32, device="cuda")
-    ws_m = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKMASS, N, H, d, ix), dtype=torch.uint8, device="cuda")
-
-    def timed(fn, reps=2):
-        out = []
-        for i in range(reps + 1):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i:
-                out.append(a.elapsed_time(b))
-        return statistics.median(out)
-
-    t_mass = timed(lambda: bsa.attn_blockmass(q, k, v, ix, wl.scale, o=o, lse=lse, mass=mass, workspace=ws_m,
-                                              stream=stream))
-    del ws_m
-    idx, cnt = bsa.losa_select(mass, wl.tau)
-    t_sel = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 10)
-    ix3 = bsa.lvsa_block_index(wl.T, frames, counts, idx, cnt)
-    ws_f = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix3), dtype=torch.uint8,
-                       device="cuda")
-    t_lvsa = timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, ix, scale=wl.scale, o=o, lse=lse, workspace=ws_f,
-                                                    stream=stream))
-    _, tcnt, _, _ = bsa.lvsa_workspace_views(ws_f, N, wl.T)
-    lvsa_tiles = int(tcnt.sum().item()) * H
-    t_both = timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, ix3, scale=wl.scale, o=o, lse=lse, workspace=ws_f,
-                                                    stream=stream))
-    status = bsa.get_device_status()
-    kept = int(cnt.sum().item())
-    flop = lambda tiles: 4 * d * tiles * 128 * 128               # noqa: E731
-    return {"workload": f"720p_14b: T=63 x P=3600 (N={N}), {H} of 40 heads, d=128, LVSA C=21 W=15 T_per=6, "
-                        "LoSA tau=0.99 inside the LVSA sets",
-            "restricted_mass_ms": t_mass, "select_us": t_sel * 1e3,
-            "lvsa_ms": t_lvsa, "lvsa_tflops_kept_tiles": flop(lvsa_tiles) / (t_lvsa / 1e3) / 1e12,
-            "intersection_ms": t_both, "intersection_tflops_kept_tiles": flop(kept) / (t_both / 1e3) / 1e12,
-            "kept_fraction_of_lvsa_tiles": kept / lvsa_tiles, "status": bsa.status_string(status)}
-
-
-def run_balanced(bsa, pool, stream, frames, counts, ix, o, lse, ws, calls=6):
-    """The balanced reading of the 6x-horizon shape (T_per = 21, 6 anchors +
-    15 window frames = C): ms per call and TFLOP/s on kept tiles over the
-    first `calls` steps (anchor phases 0..calls-1), each on its own inputs."""
-    wl = WORKLOADS["wan1.3b_6x_tper21"]
-    ms, flop, kept = [], 0, 0
-    for s in range(calls + 1):
-        bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, s, frames, counts, stream=stream)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        bsa.blocksparse_attn_fwd(*pool[s % len(pool)], ix, scale=wl.scale, o=o, lse=lse, workspace=ws, stream=stream)
-        b.record(stream)
-        torch.cuda.synchronize()
-        if s == 0:
-            continue                                  # warm-up for this index shape
-        _, tcnt, _, _ = bsa.lvsa_workspace_views(ws, wl.N, wl.T)
-        k = int(tcnt.sum().item())
-        kept += k
-        flop += 4 * wl.d * pool[0][0].shape[1] * k * 128 * 128
-        ms.append(a.elapsed_time(b))
-    status = bsa.get_device_status()
-    nB = math.ceil(wl.N / 128)
-    return {"workload": "wan1.3b_6x_tper21: as the headline shape with T_per=21 (|A(t)| = C = 21 for every t, s)",
-            "ms_per_call": statistics.median(ms), "tflops_kept_tiles": flop / (sum(ms) / 1e3) / 1e12,
-            "kept_tile_fraction": kept / calls / (nB * nB), "steps": calls, "status": bsa.status_string(status)}
-
-
 def inputs_wl(wl, rank):
     """Each rank draws its own independent problem (different seeds)."""
-    import dataclasses
     return dataclasses.replace(wl, seed_base=wl.seed_base + 100000 * rank)
 
 
@@ -591,32 +604,89 @@ def run_e2e(bsa, wl, qkv, stream, frames, counts, ix, o, lse, ws, steps, kept_ti
             "overlap": "copies on two streams beside the compute; first upload and last download not overlapped"}
 
 
-def graph_timed(fn, n, reps=5):
-    """Median ms per call of `fn` captured `n` times into one CUDA graph (so the
-    host-side cost of each call is not part of the measurement)."""
-    fn()                                   # first call on the device does its set-up outside capture
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream()
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g, stream=s):
-            for _ in range(n):
-                fn()
-    out = []
-    for i in range(reps + 1):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        g.replay()
-        b.record()
+# ------------------------------------------------------- other workloads --
+def run_configs(bsa, stream, peaks):
+    out = {}
+    for name, fn in (("tiny", lambda: lvsa_config(bsa, "tiny", stream, peaks, steps=4, graph=True)),
+                     ("wan1.3b_1x_dense", lambda: lvsa_config(bsa, "wan1.3b_1x_dense", stream, peaks, steps=5)),
+                     ("wan1.3b_1x_c11", lambda: lvsa_config(bsa, "wan1.3b_1x_c11", stream, peaks, steps=5)),
+                     ("wan1.3b_6x_tper21", lambda: lvsa_config(bsa, "wan1.3b_6x_tper21", stream, peaks, steps=6)),
+                     ("wan14b_losa", lambda: losa_config(bsa, stream, peaks)),
+                     ("720p_14b", lambda: p720_config(bsa, stream, peaks)),
+                     ("hunyuan1.5_1.5x", lambda: lvsa_config(bsa, "hunyuan1.5_1.5x", stream, peaks, steps=3,
+                                                             memory=True)),
+                     ("hunyuan1.5_2x", lambda: lvsa_config(bsa, "hunyuan1.5_2x", stream, peaks, steps=3,
+                                                           memory=True))):
+        try:
+            out[name] = fn()
+        except Exception as e:                                    # noqa: BLE001 - reported, not hidden
+            out[name] = {"error": f"{type(e).__name__}: {str(e).splitlines()[0][:200]}"}
         torch.cuda.synchronize()
-        if i:
-            out.append(a.elapsed_time(b) / n)
-    del g
-    return statistics.median(out)
+        torch.cuda.empty_cache()
+    return out
 
 
-def run_losa(bsa, rank, stream, peaks):
-    """LoSA on the Wan-2.1-14B shape: dense measuring step + mass, selection, frozen reuse."""
+def lvsa_config(bsa, name, stream, peaks, steps, graph=False, memory=False):
+    """LVSA steps 0..steps-1 of workload `name`, each on its own inputs: ms per
+    call, TFLOP/s on kept tiles and exact pairs, speed-up over the same kernel
+    on a dense index; with `memory`, the attention path's peak device memory."""
+    wl = WORKLOADS[name]
+    N, H, d = wl.N, wl.H, wl.d
+    nB = math.ceil(N / 128)
+    dev = torch.device("cuda")
+    if memory:
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()
+        base = torch.cuda.memory_allocated()
+    frames = torch.empty((wl.T, wl.T), dtype=torch.int32, device=dev)
+    counts = torch.empty((wl.T,), dtype=torch.int32, device=dev)
+    ix = bsa.lvsa_index(wl.T, frames, counts)
+    ws = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix), dtype=torch.uint8, device=dev)
+    ms, kept, exact = [], 0, 0
+    for s in range(steps):
+        qkv = inputs.workload_qkv(wl, s, device=dev)
+        o = torch.empty_like(qkv[0])
+        lse = torch.empty((H, N), dtype=torch.float32, device=dev)
+        kt, ep = lvsa_tiles(bsa, wl, s, frames, counts, ws, qkv, o, lse)
+        kept += kt
+        exact += ep
+        call = lambda: bsa.blocksparse_attn_fwd(*qkv, ix, scale=wl.scale, o=o, lse=lse, workspace=ws,  # noqa: E731
+                                                stream=stream)
+        ms.append(graph_timed(call, 20) if graph else ev_timed(call, 3, stream))
+        if s < steps - 1:
+            del qkv, o, lse
+    peak = torch.cuda.max_memory_allocated() - base if memory else None
+    dframes, dcounts = dense_frames(wl.T, dev)
+    dix = bsa.lvsa_index(wl.T, dframes, dcounts)
+    dcall = lambda: bsa.blocksparse_attn_fwd(*qkv, dix, scale=wl.scale, o=o, lse=lse, workspace=ws,  # noqa: E731
+                                             stream=stream)
+    dense_ms = graph_timed(dcall, 20) if graph else ev_timed(dcall, 2, stream)
+    status = bsa.get_device_status()
+    mean_ms = statistics.mean(ms)
+    r = rates(4 * d * H * kept * 128 * 128 / steps, 4 * d * H * exact / steps, mean_ms, peaks)
+    r.update({"workload": f"T={wl.T} x P={wl.P} (N={N}), H={H}, d={d}, LVSA C={wl.C} W={wl.W} T_per={wl.T_per}, "
+                          f"steps 0..{steps - 1} on their own inputs",
+              "steps": steps, "kept_tile_fraction": kept / steps / (nB * nB),
+              "dense_ms_per_call": dense_ms, "dense_tflops": 4 * d * H * nB * nB * 128 * 128 / (dense_ms / 1e3) / 1e12,
+              "speedup_vs_dense": dense_ms / mean_ms, "status": bsa.status_string(status)})
+    if graph:
+        r["timing"] = "20 calls replayed from one CUDA graph per step (microsecond calls)"
+    if memory:
+        qkvo = 4 * N * H * d * 2
+        r["memory"] = {"attention_path_peak_bytes": peak,
+                       "of_which_qkvo_bytes": qkvo,
+                       "workspace_bytes": ws.numel(),
+                       "dense_scores_fp32_bytes_per_head": 4 * N * N,
+                       "note": "peak device memory of the attention path alone (inputs, outputs, index, "
+                               "workspace; torch allocator); the kernels never materialise N x N scores"}
+    return r
+
+
+def losa_config(bsa, stream, peaks):
+    """LoSA on the Wan-2.1-14B shape: the dense measuring step with block mass
+    (step 0), the 99% selection, then the 39 later steps on their own
+    perturbed inputs with the frozen index; and the whole 40-step run
+    against 40 dense steps of the same kernel."""
     wl = WORKLOADS["wan14b_losa"]
     q, k, v = inputs.workload_qkv(wl, 0, device="cuda")
     N, H, d = wl.N, wl.H, wl.d
@@ -627,41 +697,117 @@ def run_losa(bsa, rank, stream, peaks):
     idx = torch.empty((H, nB, nB), dtype=torch.int32, device="cuda")
     cnt = torch.empty((H, nB), dtype=torch.int32, device="cuda")
     ws = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_DENSE_BLOCKMASS, N, H, d), dtype=torch.uint8, device="cuda")
-
-    def timed(fn, reps, batch=1):
-        """Median ms per call; `batch` calls run back to back between the events
-        (for microsecond kernels, so host-side call overhead is not timed)."""
-        out = []
-        for i in range(reps + 1):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(batch):
-                fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i:
-                out.append(a.elapsed_time(b) / batch)
-        return statistics.median(out)
-
-    t_dense = timed(lambda: bsa.attn_dense_blockmass(q, k, v, 128, wl.scale, o=o, lse=lse, mass=mass,
-                                                     workspace=ws, stream=stream), 3)
+    t_dense = ev_timed(lambda: bsa.attn_dense_blockmass(q, k, v, 128, wl.scale, o=o, lse=lse, mass=mass,
+                                                        workspace=ws, stream=stream), 3, stream)
+    del ws
     # the selection runs in microseconds: time 50 launches replayed from a CUDA graph
     t_sel = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 50)
     kept = int(cnt.sum().item())
     bix = bsa.block_index(idx, cnt)
-    qs = [inputs.workload_qkv(wl, s, device="cuda") for s in (1, 2)]
-    t_sparse = timed(lambda: bsa.blocksparse_attn_fwd(*qs[0], bix, scale=wl.scale, o=o, lse=lse, stream=stream), 5)
+    # dense forward alone (no mass), for the whole-run comparison
+    dix = bsa.block_index(*dense_block_index(H, nB))
+    t_dense_fwd = ev_timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, dix, scale=wl.scale, o=o, lse=lse,
+                                                            stream=stream), 2, stream)
+    del q, k, v
+    sparse = []
+    for s in range(1, wl.steps):
+        qs, ks, vs = inputs.workload_qkv(wl, s, device="cuda")
+        sparse.append(ev_timed(lambda: bsa.blocksparse_attn_fwd(qs, ks, vs, bix, scale=wl.scale, o=o, lse=lse,
+                                                                stream=stream), 1, stream, warm=1 if s == 1 else 0))
+        del qs, ks, vs
     status = bsa.get_device_status()
-    dense_flop = 4 * d * H * N * N
     sel_bytes = mass.numel() * 4 + idx.numel() * 4 + cnt.numel() * 4
-    return {"workload": "wan14b_losa: T=21 x P=1560 (N=32760), H=40, d=128, block 128, tau=0.99",
-            "dense_blockmass_ms": t_dense,
-            "dense_fwd_tflops_equiv": dense_flop / (t_dense / 1e3) / 1e12,
-            "select_us": t_sel * 1e3, "select_gbs": sel_bytes / (t_sel / 1e3) / 1e9,
-            "select_frac_of_hbm": sel_bytes / (t_sel / 1e3) / 1e9 / peaks["hbm"],
-            "kept_block_fraction": kept / (H * nB * nB),
-            "sparse_ms_per_call": t_sparse,
-            "sparse_tflops_kept_blocks": 4 * d * kept * 128 * 128 / (t_sparse / 1e3) / 1e12,
+    dense_flop = 4 * d * H * N * N
+    run_ms = t_dense + t_sel + sum(sparse)
+    r = rates(4 * d * kept * 128 * 128, 4 * d * kept * 128 * 128, statistics.mean(sparse), peaks)
+    r.pop("tflops_exact_pairs")
+    r.pop("frac_exact_of_bf16_burst")
+    r.update({"workload": "wan14b_losa: T=21 x P=1560 (N=32760), H=40, d=128, block 128, tau=0.99; step 0 dense "
+                          "measuring step, steps 1..39 frozen index on their own perturbed inputs",
+              "ms_per_call": statistics.mean(sparse), "ms_per_call_median": statistics.median(sparse),
+              "frozen_steps": len(sparse),
+              "dense_blockmass_ms": t_dense, "dense_blockmass_tflops_equiv": dense_flop / (t_dense / 1e3) / 1e12,
+              "dense_fwd_ms": t_dense_fwd, "dense_fwd_tflops": dense_flop / (t_dense_fwd / 1e3) / 1e12,
+              "select_us": t_sel * 1e3, "select_gbs": sel_bytes / (t_sel / 1e3) / 1e9,
+              "select_frac_of_hbm": sel_bytes / (t_sel / 1e3) / 1e9 / peaks["hbm"],
+              "kept_block_fraction": kept / (H * nB * nB),
+              "run_40_steps_ms": run_ms, "dense_40_steps_ms": 40 * t_dense_fwd,
+              "run_speedup_vs_dense": 40 * t_dense_fwd / run_ms,
+              "status": bsa.status_string(status)})
+    return r
+
+
+def dense_block_index(H, nB):
+    idx = torch.arange(nB, dtype=torch.int32, device="cuda").repeat(H, nB, 1).contiguous()
+    cnt = torch.full((H, nB), nB, dtype=torch.int32, device="cuda")
+    return idx, cnt
+
+
+def p720_config(bsa, stream, peaks):
+    """720p long video with 14B heads (T=63 x P=3600, all 40 heads): LVSA
+    steps; LoSA alone (dense measuring step, selection, frozen-index step);
+    LoSA inside LVSA (restricted measuring step, selection, intersection
+    step)."""
+    wl = WORKLOADS["720p_14b"]
+    N, H, d = wl.N, wl.H, wl.d
+    nB = math.ceil(N / 128)
+    q, k, v = inputs.workload_qkv(wl, 0, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((H, N), dtype=torch.float32, device="cuda")
+    frames = torch.empty((wl.T, wl.T), dtype=torch.int32, device="cuda")
+    counts = torch.empty((wl.T,), dtype=torch.int32, device="cuda")
+    ix = bsa.lvsa_index(wl.T, frames, counts)
+    ws = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix), dtype=torch.uint8, device="cuda")
+    lv_ms, kept, exact = [], 0, 0
+    for s in range(3):                                  # three anchor phases on the same inputs
+        kt, ep = lvsa_tiles(bsa, wl, s, frames, counts, ws, (q, k, v), o, lse)
+        kept += kt
+        exact += ep
+        lv_ms.append(ev_timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, ix, scale=wl.scale, o=o, lse=lse,
+                                                               workspace=ws, stream=stream), 1, stream, warm=0))
+    lvsa = rates(4 * d * H * kept * 128 * 128 / 3, 4 * d * H * exact / 3, statistics.mean(lv_ms), peaks)
+    lvsa["steps"] = 3
+    # LoSA inside LVSA at step 0: restricted measuring step, selection, intersection step
+    bsa.lvsa_build_index(wl.T, wl.T_per, wl.W, wl.C, 0, frames, counts)
+    mass = torch.empty((H, nB, nB), dtype=torch.float32, device="cuda")
+    wsm = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKMASS, N, H, d, ix), dtype=torch.uint8, device="cuda")
+    t_rmass = ev_timed(lambda: bsa.attn_blockmass(q, k, v, ix, wl.scale, o=o, lse=lse, mass=mass, workspace=wsm,
+                                                  stream=stream), 1, stream)
+    idx = torch.empty((H, nB, nB), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((H, nB), dtype=torch.int32, device="cuda")
+    t_sel_r = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 5)
+    kept_r = int(cnt.sum().item())
+    lvsa0_tiles = lvsa_tiles(bsa, wl, 0, frames, counts, ws, (q, k, v), o, lse)[0]
+    ix3 = bsa.lvsa_block_index(wl.T, frames, counts, idx, cnt)
+    ws3 = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix3), dtype=torch.uint8,
+                      device="cuda")
+    t_both = ev_timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, ix3, scale=wl.scale, o=o, lse=lse, workspace=ws3,
+                                                       stream=stream), 2, stream)
+    del ws3
+    # LoSA alone on the same inputs: dense measuring step (head passes in a 4 GiB workspace), selection, sparse step
+    t_dmass = ev_timed(lambda: bsa.attn_dense_blockmass(q, k, v, 128, wl.scale, o=o, lse=lse, mass=mass,
+                                                        workspace=wsm, stream=stream), 1, stream)
+    del wsm
+    t_sel = graph_timed(lambda: bsa.losa_select(mass, wl.tau, idx=idx, cnt=cnt), 5)
+    kept_l = int(cnt.sum().item())
+    bix = bsa.block_index(idx, cnt)
+    t_losa = ev_timed(lambda: bsa.blocksparse_attn_fwd(q, k, v, bix, scale=wl.scale, o=o, lse=lse, stream=stream),
+                      2, stream)
+    status = bsa.get_device_status()
+    sel_bytes = mass.numel() * 8 + cnt.numel() * 4
+    fl = lambda tiles: 4 * d * tiles * 128 * 128                  # noqa: E731
+    dense_flop = 4 * d * H * N * N
+    return {"workload": f"720p_14b: T=63 x P=3600 (N={N}), H={H}, d=128, LVSA C=21 W=15 T_per=6; LoSA tau=0.99",
+            "lvsa": lvsa,
+            "losa_in_lvsa": {"restricted_mass_ms": t_rmass, "select_us": t_sel_r * 1e3,
+                             "select_gbs": sel_bytes / (t_sel_r / 1e3) / 1e9,
+                             "intersection_ms": t_both,
+                             "intersection_tflops_kept_tiles": fl(kept_r) / (t_both / 1e3) / 1e12,
+                             "kept_fraction_of_lvsa_tiles": kept_r / (lvsa0_tiles * H)},
+            "losa": {"dense_blockmass_ms": t_dmass, "dense_blockmass_tflops_equiv": dense_flop / (t_dmass / 1e3) / 1e12,
+                     "select_us": t_sel * 1e3, "select_gbs": sel_bytes / (t_sel / 1e3) / 1e9,
+                     "sparse_ms": t_losa, "sparse_tflops_kept_blocks": fl(kept_l) / (t_losa / 1e3) / 1e12,
+                     "kept_block_fraction": kept_l / (H * nB * nB)},
             "status": bsa.status_string(status)}
 
 
@@ -669,7 +815,6 @@ def run_select_only():
     """Profiling case for the LoSA selection alone, small on the device: block
     masses from a 4-head dense measuring step on the Wan-2.1-14B shape, tiled
     to that workload's 40 heads (10,240 rows of 256 key blocks)."""
-    import dataclasses
     import block_sparse_attention_lvsa_b200.binding as bsa
     wl = dataclasses.replace(WORKLOADS["wan14b_losa"], H=4)
     q, k, v = inputs.workload_qkv(wl, 0, device="cuda")
@@ -688,25 +833,32 @@ def run_select_only():
                       "us": a.elapsed_time(b) * 1e3, "status": bsa.status_string(bsa.get_device_status())}))
 
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--cpu-rows", type=int, default=16384)
+    ap.add_argument("--workload", choices=LVSA_WORKLOADS, default=WORKLOAD,
+                    help="LVSA workload of the timed steps (default: the headline 6x-horizon shape)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' extra keys")
     ap.add_argument("--heads", type=int, default=0, help="profiling only: override the head count")
     ap.add_argument("--main-only", action="store_true", help="profiling only: timed LVSA steps, nothing else")
     ap.add_argument("--select-only", action="store_true", help="profiling only: the LoSA selection, small case")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: independent replicas (weak scaling) or one problem split by heads (strong)")
-    args = ap.parse_args()
+    argv = sys.argv[1:] if argv is None else argv
+    args = ap.parse_args(argv)
     if args.select_only:
         run_select_only()
-        return
+        return 0
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus, argv)
     rank, world, local = dist_init(args.gpus)
     try:
         if args.impl == "reference":
@@ -717,7 +869,8 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

@@ -63,6 +63,19 @@ WORKLOADS = {
     "wan14b_losa": Workload("wan14b_losa", T=21, P=1560, H=40, d=128,
                             block=128, tau=0.99, steps=40, locality=2.0,
                             perturb=0.1, seed_base=4000),
+    # HunyuanVideo-1.5-shaped long video at 1.5x and 2x its 129-frame
+    # training horizon (193 and 257 frames).  The LVSA explainer names the
+    # model, the horizons and the memory check (section 4) but not its
+    # latent shape; readings: a causal video VAE with 4x temporal
+    # compression gives 1 + (frames - 1) / 4 latent frames (33 at the
+    # training horizon, 49 and 65 here), 720p with 16x spatial compression
+    # and no further patching gives 80 x 45 = 3600 tokens per frame, 16 heads
+    # of 128 channels; budget C = the 33-frame training horizon (as C = 21
+    # for Wan), T_per = 6 as in the Wan workloads, W = C - |G_s|.
+    "hunyuan1.5_1.5x": Workload("hunyuan1.5_1.5x", T=49, P=3600, H=16, d=128, C=33, W=24,
+                                T_per=6, steps=50, seed_base=6000),
+    "hunyuan1.5_2x": Workload("hunyuan1.5_2x", T=65, P=3600, H=16, d=128, C=33, W=22,
+                              T_per=6, steps=50, seed_base=7000),
     # 720p long video with 14B heads, LVSA plus LoSA selection
     "720p_14b": Workload("720p_14b", T=63, P=3600, H=40, d=128, C=21, W=15,
                          T_per=6, steps=40, block=128, tau=0.99, locality=2.0,

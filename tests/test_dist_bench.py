@@ -41,3 +41,38 @@ def test_two_rank_reductions():
     assert out[0][0] == out[1][0] == 11.0          # max over ranks
     assert out[0][1] == out[1][1] == 3.0           # sum over ranks
     assert out[0][2] != out[1][2]                  # independent problems per rank
+
+
+def _bench(args, env_extra=None, timeout=600):
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR",
+                                                            "MASTER_PORT")}
+    env.update(env_extra or {})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, capture_output=True, text=True,
+                          timeout=timeout, env=env, cwd=root)
+
+
+@pytest.mark.timeout(900)
+def test_gpus_two_starts_two_ranks():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself (here on
+    CPU with gloo, through the oracle arm on the tiny workload): the line
+    reports n_gpus 2 and only rank 0 prints it."""
+    import json
+    r = _bench(["--gpus", "2", "--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+    assert lines[0]["cpu_baseline"]["cores"] >= 1
+
+
+@pytest.mark.timeout(300)
+def test_gpus_mismatch_refused():
+    """Under a launcher whose world size differs from --gpus the run stops
+    with an error instead of reporting the wrong number of GPUs."""
+    r = _bench(["--gpus", "2", "--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+               env_extra={"WORLD_SIZE": "1", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode != 0
+    assert "WORLD_SIZE" in r.stderr

@@ -9,7 +9,8 @@ from block_sparse_attention_lvsa_b200.workloads import WORKLOADS
 
 pytestmark = pytest.mark.gpu
 
-LVSA_WL = ["tiny", "wan1.3b_1x_dense", "wan1.3b_1x_c11", "wan1.3b_6x", "wan1.3b_6x_tper21", "720p_14b"]
+LVSA_WL = ["tiny", "wan1.3b_1x_dense", "wan1.3b_1x_c11", "wan1.3b_6x", "wan1.3b_6x_tper21", "720p_14b",
+           "hunyuan1.5_1.5x", "hunyuan1.5_2x"]
 
 
 @pytest.fixture(scope="module")
@@ -115,7 +116,8 @@ def test_tiles_small_random(bsa):
 
 
 @pytest.mark.parametrize("name,steps", [("tiny", [0, 1, 2, 3]), ("wan1.3b_1x_c11", [0, 3]),
-                                        ("wan1.3b_6x", [0, 5]), ("720p_14b", [0])])
+                                        ("wan1.3b_6x", [0, 5]), ("720p_14b", [0]),
+                                        ("hunyuan1.5_1.5x", [0, 1]), ("hunyuan1.5_2x", [0, 5])])
 def test_tiles_workloads(bsa, name, steps):
     wl = WORKLOADS[name]
     nB = -(-wl.N // 128)

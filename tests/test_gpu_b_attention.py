@@ -176,3 +176,9 @@ def test_window_reading(bsa, name, s):
 
 def test_720p_lvsa_full_size(bsa):
     sampled_lvsa(bsa, WORKLOADS["720p_14b"], 0, 128, [0, 39], 50)
+
+
+@pytest.mark.parametrize("name,s", [("hunyuan1.5_1.5x", 0), ("hunyuan1.5_2x", 0), ("hunyuan1.5_2x", 5)])
+def test_hunyuan_horizons_full_size(bsa, name, s):
+    """HunyuanVideo-1.5-shaped long video at 1.5x and 2x its training horizon."""
+    sampled_lvsa(bsa, WORKLOADS[name], s, 128, [0, 15], 55 + s)
