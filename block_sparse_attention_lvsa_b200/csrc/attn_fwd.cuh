@@ -225,14 +225,6 @@ __device__ __forceinline__ void apply_mask128(float* s, const uint32_t (&mw)[4])
     if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
 }
 
-// Of every 8 column pairs of an unmasked tile, kPolyCols / 16 take
-// exp2_poly3_x2 on the FMA pipe and the rest ex2 on MUFU (masked tiles stay on
-// MUFU: the polynomial does not give exactly 0 for a masked score).  Off:
-// with the warp-wide MMA issue and the register split, 16 and 32 columns
-// measured the same as 0 (39.68 / 39.65 vs 39.70 ms): a softmax warp's
-// exponential phase is bound by its own instruction stream, not by MUFU.
-constexpr int kPolyCols = 0;
-
 // exp2(s * sl2 - m) for one 128-score row; P (bf16 pairs) packed in place
 // into sr[0..63] (pair j overwrites sr[j] only after elements 2j, 2j+1 >= j
 // are read).  Returns the row sum of the float32 values.
@@ -260,49 +252,9 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x of a packed pair on the FMA pipe, for x <= ~10 (inputs below -125
-// give ~2^-125, not 0; the clamp keeps the exponent field of the result
-// positive).
-// x = j + f with j = round(x) (adding and removing 1.5 * 2^23 rounds to the
-// nearest integer) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted
-// by Remez exchange for minimum relative error on [-1/2, 1/2] (max relative
-// error 7.5e-5, below the bf16 half-ulp of 2^-9 that P is rounded to); 2^j is
-// added to the exponent field as an integer (the exponent of t's bit pattern
-// cancels: (0x4B400000 << 23) == 0 mod 2^32).  The adds and the polynomial
-// run as f32x2 instructions (same per-lane rounding), the clamp and the
-// exponent-field add per lane.  Available to take part of the exponentials
-// of unmasked tiles off the MUFU unit (kPolyCols columns).
-__device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t xp) {
-  float a, b;
-  f2unpack(xp, a, b);
-  xp = f2pack(fmaxf(a, -125.0f), fmaxf(b, -125.0f));
-  const uint64_t t = fadd2(xp, f2pack(12582912.0f, 12582912.0f));
-  const uint64_t j = fadd2(t, f2pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = ffma2(j, f2pack(-1.0f, -1.0f), xp);
-  uint64_t q = ffma2(f2pack(0.0551716685295105f, 0.0551716685295105f), f,
-                     f2pack(0.2426111251115799f, 0.2426111251115799f));
-  q = ffma2(q, f, f2pack(0.6932609677314758f, 0.6932609677314758f));
-  q = ffma2(q, f, f2pack(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, t0, t1;
-  f2unpack(q, q0, q1);
-  f2unpack(t, t0, t1);
-  return f2pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
-                __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
-}
-
-// column pair j (columns 2j, 2j+1) of an unmasked tile takes the polynomial:
-// NPOLY / 16 of every 8 pairs
-template <int NPOLY>
-__device__ __forceinline__ constexpr bool poly_pair(int j) {
-  return (j & 7) < NPOLY / 16;
-}
-
 // P of keys 0..63 (sr[0..31]) goes to TMEM as soon as it is formed, keys
 // 64..127 after the loop; the caller waits for both stores
 // (tmem_wait_st) before signalling P ready.
-constexpr bool kSplitPStore = true;
-
-template <int NPOLY>
 __device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use, uint32_t tP) {
   const uint64_t sl2p = f2pack(sl2, sl2), nm = f2pack(-m_use, -m_use);
   uint64_t acc01 = f2pack(0.f, 0.f), acc23 = f2pack(0.f, 0.f);
@@ -310,21 +262,11 @@ __device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, floa
   for (int c = 0; c < 128; c += 4) {
     const uint64_t x01 = ffma2(f2pack(s[c], s[c + 1]), sl2p, nm);
     const uint64_t x23 = ffma2(f2pack(s[c + 2], s[c + 3]), sl2p, nm);
-    uint64_t e01, e23;
-    if (poly_pair<NPOLY>(c / 2)) {
-      e01 = exp2_poly3_x2(x01);
-    } else {
-      float x0, x1;
-      f2unpack(x01, x0, x1);
-      e01 = f2pack(ex2_approx(x0), ex2_approx(x1));
-    }
-    if (poly_pair<NPOLY>(c / 2 + 1)) {
-      e23 = exp2_poly3_x2(x23);
-    } else {
-      float x2, x3;
-      f2unpack(x23, x2, x3);
-      e23 = f2pack(ex2_approx(x2), ex2_approx(x3));
-    }
+    float x0, x1, x2, x3;
+    f2unpack(x01, x0, x1);
+    f2unpack(x23, x2, x3);
+    const uint64_t e01 = f2pack(ex2_approx(x0), ex2_approx(x1));
+    const uint64_t e23 = f2pack(ex2_approx(x2), ex2_approx(x3));
     acc01 = fadd2(acc01, e01);
     acc23 = fadd2(acc23, e23);
     float e0, e1, e2, e3;
@@ -332,14 +274,9 @@ __device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, floa
     f2unpack(e23, e2, e3);
     sr[c / 2] = pack_bf16x2(e0, e1);
     sr[c / 2 + 1] = pack_bf16x2(e2, e3);
-    if (kSplitPStore && c == 60) tmem_st_x32_async(tP, sr);
+    if (c == 60) tmem_st_x32_async(tP, sr);
   }
-  if (kSplitPStore) {
-    tmem_st_x32_async(tP + 32, sr + 32);
-  } else {
-    tmem_st_x32_async(tP, sr);
-    tmem_st_x32_async(tP + 32, sr + 32);
-  }
+  tmem_st_x32_async(tP + 32, sr + 32);
   float r0, r1, r2, r3;
   f2unpack(acc01, r0, r1);
   f2unpack(acc23, r2, r3);
@@ -649,10 +586,8 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
           }
         }
-        // p = exp2(s * scale * log2e - m), P packed in place (the tile's flag is
-        // the same for the whole group: no divergence)
-        const float rsum =
-            part ? row_exp_pack<0>(s, sr, p.sl2, m_use, tS) : row_exp_pack<kPolyCols>(s, sr, p.sl2, m_use, tS);
+        // p = exp2(s * scale * log2e - m), P packed in place
+        const float rsum = row_exp_pack(s, sr, p.sl2, m_use, tS);
         tmem_wait_st();
         if constexpr (MASS) {
           // this tile's share of the row's mass, log2, before normalisation

@@ -110,7 +110,7 @@ def test_losa_select_bitexact_on_gpu_mass(bsa, losa_step0):
     assert 0.0 < kept < 1.0
 
 
-@pytest.mark.parametrize("nKB", [1, 2, 7, 128, 256, 257, 1772, 8192])
+@pytest.mark.parametrize("nKB", [1, 2, 7, 128, 256, 257, 700, 1772, 3000, 8192])
 def test_losa_select_random(bsa, nKB):
     rng = np.random.default_rng(nKB)
     H, nQB = 2, 3
