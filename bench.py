@@ -499,10 +499,11 @@ def run_b200(args, rank, world, local):
 
 
 # DRAM bytes (read + write) per launch of the attention kernel at the full
-# 12-head workload, from an ncu capture of the 4-head case of the same
-# workload scaled by 12/4 (traffic grows with the number of heads); None
-# until the counters are taken on the current kernel.
-TRAFFIC_PER_LAUNCH = None
+# 12-head workload: the ncu capture of the 4-head case of the same workload
+# (652.7 MB read + 192.1 MB written, step-0 index) scaled by 12/4 (traffic
+# grows with the number of heads).  Must be re-measured (or set to None)
+# whenever the kernel changes.
+TRAFFIC_PER_LAUNCH = 2.534e9
 
 
 def run_gather(o, lse, H, world, reps=3):
