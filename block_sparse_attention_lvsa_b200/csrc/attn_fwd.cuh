@@ -33,6 +33,10 @@
 // Tensor-core order per key tile i (ping-pong between the two groups):
 //   S_0(i) = Q_0 K_i^T,  O_1 += P_1(i-1) V_{i-1},  S_1(i) = Q_1 K_i^T,
 //   O_0 += P_0(i) V_i
+// Each PV goes out in two halves of 64 keys: the softmax signals once after
+// storing P of the first 64 keys and again after the rest, so the first
+// half of the product runs while the softmax still computes the second half
+// of the exponentials.
 // While group 0 turns S_0(i) into P_0(i) the tensor core runs O_1 and S_1,
 // and the other way round.  MMAs issued by one thread execute in order, so
 // S_x(i+1) (issued after O_x's PV) cannot overwrite P_x(i) before it is read,
@@ -120,7 +124,8 @@ enum : int {
   B_SFULL = B_VEMPTY + kVStages,      // [group]
   B_PFULL = B_SFULL + 2,              // [group]
   B_PVDONE = B_PFULL + 2,             // [group]
-  B_FINAL = B_PVDONE + 2,
+  B_PLO = B_PVDONE + 2,               // [group] first 64 keys of P stored
+  B_FINAL = B_PLO + 2,
   B_COUNT = B_FINAL + 1
 };
 static_assert(B_COUNT <= 32, "barrier slots");
@@ -252,10 +257,12 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// P of keys 0..63 (sr[0..31]) goes to TMEM as soon as it is formed, keys
-// 64..127 after the loop; the caller waits for both stores
-// (tmem_wait_st) before signalling P ready.
-__device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use, uint32_t tP) {
+// P of keys 0..63 (sr[0..31]) goes to TMEM as soon as it is formed and is
+// signalled on `plo_bar` (the PV of those keys can start), keys 64..127 after
+// the loop; the caller waits for that store (tmem_wait_st) before signalling
+// the whole P ready.
+__device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, float sl2, float m_use, uint32_t tP,
+                                              uint32_t plo_bar, int lane) {
   const uint64_t sl2p = f2pack(sl2, sl2), nm = f2pack(-m_use, -m_use);
   uint64_t acc01 = f2pack(0.f, 0.f), acc23 = f2pack(0.f, 0.f);
 #pragma unroll
@@ -274,7 +281,13 @@ __device__ __forceinline__ float row_exp_pack(const float* s, uint32_t* sr, floa
     f2unpack(e23, e2, e3);
     sr[c / 2] = pack_bf16x2(e0, e1);
     sr[c / 2 + 1] = pack_bf16x2(e2, e3);
-    if (c == 60) tmem_st_x32_async(tP, sr);
+    if (c == 60) {
+      tmem_st_x32_async(tP, sr);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(plo_bar);
+    }
   }
   tmem_st_x32_async(tP + 32, sr + 32);
   float r0, r1, r2, r3;
@@ -346,6 +359,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int x = 0; x < 2; ++x) mbar_init(bar(B_SFULL + x), 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(B_PFULL + x), 4);
+      mbar_init(bar(B_PLO + x), 4);
       mbar_init(bar(B_PVDONE + x), 1);
     }
     mbar_init(bar(B_FINAL), 1);
@@ -436,21 +450,26 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (bar2 >= 0) tc_commit2_warp(bar(B_SFULL + sb), bar(bar2));
         else tc_commit_warp(bar(B_SFULL + sb));
       };
-      // wait until V of key tile `vit` and P_x of the group's c-th tile are in place
+      // wait until V of key tile `vit` and P_x of the first 64 keys of the
+      // group's c-th tile are in place
       auto pv_ready = [&](int x, int vit, int c) -> bool {
         if (!mbar_wait_warp(bar(B_VFULL + vit % kVStages), (vit / kVStages) & 1, limit)) return false;
-        if (!mbar_wait_warp(bar(B_PFULL + x), c & 1, limit)) return false;
+        if (!mbar_wait_warp(bar(B_PLO + x), c & 1, limit)) return false;
         tc_fence_after();
         return true;
       };
-      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major); completion
+      // O_x += P_x V (P_x from TMEM, V from shared memory, MN-major): the first
+      // 64 keys at once, the other 64 once the softmax has stored them (an
+      // expired wait skips them; the status word already says so); completion
       // on PVDONE + x (and, when given, on a second barrier)
       auto pv = [&](int x, int vit, int c, int bar2) {
         const uint64_t dv = desc64(sw128_desc(base + L::kV + (vit % kVStages) * L::kTile, L::kBox, 1024));
         const uint32_t tO = tbase + L::kTmemO + x * D;
         const uint32_t tP = tbase + x * 128;
         mma4_ts_warp(tO, tP, dv, kIdescPV, c > 0 ? 1u : 0u);     // keys 0..63
-        mma4_ts_warp(tO, tP + 32, dv + 512, kIdescPV, 1u);       // keys 64..127
+        const bool full = mbar_wait_warp(bar(B_PFULL + x), c & 1, limit);
+        tc_fence_after();
+        if (full) mma4_ts_warp(tO, tP + 32, dv + 512, kIdescPV, 1u);       // keys 64..127
         if (bar2 >= 0) tc_commit2_warp(bar(B_PVDONE + x), bar(bar2));
         else tc_commit_warp(bar(B_PVDONE + x));
       };
@@ -587,7 +606,7 @@ attn_tile_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
         }
         // p = exp2(s * scale * log2e - m), P packed in place
-        const float rsum = row_exp_pack(s, sr, p.sl2, m_use, tS);
+        const float rsum = row_exp_pack(s, sr, p.sl2, m_use, tS, bar(B_PLO + x), lane);
         tmem_wait_st();
         if constexpr (MASS) {
           // this tile's share of the row's mass, log2, before normalisation
