@@ -37,6 +37,7 @@ import subprocess
 import sys
 import tempfile
 import time
+import warnings
 
 import torch
 
@@ -300,10 +301,14 @@ def graph_timed(fn, n, reps=5):
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
-    with torch.cuda.stream(s):
-        with torch.cuda.graph(g, stream=s):
-            for _ in range(n):
-                fn()
+    with warnings.catch_warnings():
+        # a call that launches on a stream other than the capturing one leaves the graph
+        # empty and its replay times nothing: make that an error, not a number
+        warnings.filterwarnings("error", message=".*CUDA Graph is empty.*")
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(n):
+                    fn()
     out = []
     for i in range(reps + 1):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -500,10 +505,10 @@ def run_b200(args, rank, world, local):
 
 # DRAM bytes (read + write) per launch of the attention kernel at the full
 # 12-head workload: the ncu capture of the 4-head case of the same workload
-# (652.7 MB read + 192.1 MB written, step-0 index) scaled by 12/4 (traffic
+# (666.9 MB read + 192.4 MB written, step-0 index) scaled by 12/4 (traffic
 # grows with the number of heads).  Must be re-measured (or set to None)
 # whenever the kernel changes.
-TRAFFIC_PER_LAUNCH = 2.534e9
+TRAFFIC_PER_LAUNCH = 2.578e9
 
 
 def run_gather(o, lse, H, world, reps=3):
@@ -644,6 +649,7 @@ def lvsa_config(bsa, name, stream, peaks, steps, graph=False, memory=False):
     ix = bsa.lvsa_index(wl.T, frames, counts)
     ws = torch.empty(bsa.workspace_bytes(bsa.BSA_OP_BLOCKSPARSE_FWD, N, H, d, ix), dtype=torch.uint8, device=dev)
     ms, kept, exact = [], 0, 0
+    launch_stream = None if graph else stream      # under graph capture: the capturing (current) stream
     for s in range(steps):
         qkv = inputs.workload_qkv(wl, s, device=dev)
         o = torch.empty_like(qkv[0])
@@ -652,7 +658,7 @@ def lvsa_config(bsa, name, stream, peaks, steps, graph=False, memory=False):
         kept += kt
         exact += ep
         call = lambda: bsa.blocksparse_attn_fwd(*qkv, ix, scale=wl.scale, o=o, lse=lse, workspace=ws,  # noqa: E731
-                                                stream=stream)
+                                                stream=launch_stream)
         ms.append(graph_timed(call, 20) if graph else ev_timed(call, 3, stream))
         if s < steps - 1:
             del qkv, o, lse
@@ -660,7 +666,7 @@ def lvsa_config(bsa, name, stream, peaks, steps, graph=False, memory=False):
     dframes, dcounts = dense_frames(wl.T, dev)
     dix = bsa.lvsa_index(wl.T, dframes, dcounts)
     dcall = lambda: bsa.blocksparse_attn_fwd(*qkv, dix, scale=wl.scale, o=o, lse=lse, workspace=ws,  # noqa: E731
-                                             stream=stream)
+                                             stream=launch_stream)
     dense_ms = graph_timed(dcall, 20) if graph else ev_timed(dcall, 2, stream)
     status = bsa.get_device_status()
     mean_ms = statistics.mean(ms)
