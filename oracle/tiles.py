@@ -10,15 +10,7 @@ Definitions (element level, rows and columns restricted to [0, N)):
   * key tile kt is KEPT for query tile qt iff some q in qt, k in kt has
     frame(k) in A(frame(q));
   * a kept tile is PARTIAL iff some pair (q, k) with q in qt, k in kt, both
-    < N, is not allowed, or the tile reaches past N (its last column >= N);
-  * a half (the first or the last tile/2 columns) of a kept tile is DEAD iff
-    no pair (q, k) with q in qt, k in that half, both < N, is allowed (a half
-    lying wholly past N is dead).  Such a half contributes nothing to any row
-    of the tile, so a kernel may skip its products.  A kept tile has at most
-    one dead half, and a tile with a dead half is partial.
-
-The flag of a kept tile is PARTIAL | 2 * (first half dead) | 4 * (last half
-dead).
+    < N, is not allowed, or the tile reaches past N (its last column >= N).
 
 Because the frames of the rows of a tile form a contiguous range (and so do
 the frames of its columns), the tests of "some pair" / "all pairs" reduce to
@@ -40,8 +32,7 @@ TILE = 128
 
 def kept_tiles(A: List[List[int]], T: int, N: int, tile: int = TILE,
                qtiles=None) -> Tuple[List[List[int]], List[List[int]]]:
-    """Per query tile: ascending kept key tiles and their flags (partial bit 1,
-    first-half-dead bit 2, last-half-dead bit 4).
+    """Per query tile: ascending kept key tiles and their partial flags (0/1).
 
     ``qtiles`` (optional) restricts the evaluation to those query tiles; the
     returned lists then follow that order.
@@ -64,12 +55,7 @@ def kept_tiles(A: List[List[int]], T: int, N: int, tile: int = TILE,
             if sub.any():
                 row_i.append(kt)
                 partial = (not sub.all()) or ((kt + 1) * tile > N)
-                dead = []
-                for half in range(2):
-                    h_lo = k_lo + half * (tile // 2)
-                    h_hi = min(h_lo + tile // 2, N) - 1
-                    dead.append(h_lo > h_hi or not M[fq_lo:fq_hi + 1, h_lo // P:h_hi // P + 1].any())
-                row_f.append(int(partial) | 2 * int(dead[0]) | 4 * int(dead[1]))
+                row_f.append(int(partial))
         idx.append(row_i)
         flg.append(row_f)
     return idx, flg
@@ -89,12 +75,7 @@ def kept_tiles_bruteforce(A: List[List[int]], T: int, N: int, tile: int = TILE):
             blk = mask[rows, cols]
             if blk.any():
                 ri.append(kt)
-                f = int((not blk.all()) or (kt + 1) * tile > N)
-                for half in range(2):
-                    hc = mask[rows, kt * tile + half * (tile // 2):min(kt * tile + (half + 1) * (tile // 2), N)]
-                    if not hc.any():                      # empty (past N) or no allowed pair
-                        f |= 2 << half
-                rf.append(f)
+                rf.append(int((not blk.all()) or (kt + 1) * tile > N))
         idx.append(ri)
         flg.append(rf)
     return idx, flg

@@ -192,40 +192,6 @@ def check_tiles_vs_bruteforce(tiles, lvsa):
         assert tiles.kept_tiles(A, 8, 512) == tiles.kept_tiles_bruteforce(A, 8, 512)
 
 
-def check_tiles_half_frames(tiles, trials=6):
-    """Closed form with P = 64 tokens per frame: a 128-tile holds exactly two
-    frames and each 64-key half exactly one, so for query tile qt (frames
-    2qt, 2qt+1) and key tile kt (frames 2kt, 2kt+1), with U the union and X
-    the intersection of A over the two query frames: kt is kept iff 2kt or
-    2kt+1 is in U; partial iff one of them is not in X; half h is dead iff
-    2kt+h is not in U."""
-    rng = np.random.default_rng(11)
-    T, P = 8, 64
-    for _ in range(trials):
-        A = random_allowed(T, rng)
-        idx, flg = tiles.kept_tiles(A, T, T * P)
-        for qt in range(T // 2):
-            U = set(A[2 * qt]) | set(A[2 * qt + 1])
-            X = set(A[2 * qt]) & set(A[2 * qt + 1])
-            want_i, want_f = [], []
-            for kt in range(T // 2):
-                fr = (2 * kt, 2 * kt + 1)
-                if fr[0] in U or fr[1] in U:
-                    want_i.append(kt)
-                    f = int(not (fr[0] in X and fr[1] in X))
-                    f |= 2 * int(fr[0] not in U) | 4 * int(fr[1] not in U)
-                    want_f.append(f)
-            assert idx[qt] == want_i and flg[qt] == want_f, (qt, A)
-    # a last tile of at most 64 keys: its upper half lies past N and is dead
-    for T, P in ((4, 80), (3, 100), (1, 64), (2, 96)):
-        N = T * P
-        A = [list(range(T)) for _ in range(T)]
-        idx, flg = tiles.kept_tiles(A, T, N)
-        nB = -(-N // 128)
-        assert all(r == list(range(nB)) for r in idx)
-        assert all(f == [0] * (nB - 1) + [1 | 4] for f in flg), (T, P)
-
-
 # ------------------------------------------------------------ attention ---
 def sdpa_f64(q, k, v, scale, mask=None):
     """torch CPU float64 scaled_dot_product_attention, [N,H,d] layout in and out."""

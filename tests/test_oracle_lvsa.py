@@ -47,10 +47,6 @@ def test_tiles_bruteforce():
     pins.check_tiles_vs_bruteforce(tiles, lvsa)
 
 
-def test_tiles_half_frames_closed_form():
-    pins.check_tiles_half_frames(tiles)
-
-
 def test_tiles_dense_full():
     # every tile kept; only tiles reaching past N are partial
     A, _ = lvsa.attended_frames(21, 5, 7, 21, 0)

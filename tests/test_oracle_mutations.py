@@ -155,60 +155,6 @@ def test_tiles_partial_flag_caught():
     assert fails(pins.check_tiles_vs_bruteforce, m, lvsa)
 
 
-def _mutant_dead_halves(rule):
-    """kept_tiles with the dead-half bits recomputed by `rule(sub_half, h_lo, h_hi)`."""
-    m = clone(tiles)
-
-    def kept(A, T, N, tile=128, qtiles=None):
-        idx, flg = tiles.kept_tiles(A, T, N, tile, qtiles)
-        P = N // T
-        M = lvsa.allowed_frames_matrix(A, T)
-        out = []
-        for qt, (ri, rf) in zip(range(len(idx)) if qtiles is None else qtiles, zip(idx, flg)):
-            fq_lo, fq_hi = qt * tile // P, (min((qt + 1) * tile, N) - 1) // P
-            row = []
-            for kt, f in zip(ri, rf):
-                f &= 1
-                for half in range(2):
-                    h_lo = kt * tile + half * (tile // 2)
-                    h_hi = min(h_lo + tile // 2, N) - 1
-                    sub = M[fq_lo:fq_hi + 1, h_lo // P:max(h_hi, h_lo) // P + 1]
-                    if rule(sub, h_lo, h_hi):
-                        f |= 2 << half
-                row.append(f)
-            out.append(row)
-        return idx, out
-    m.kept_tiles = kept
-    return m
-
-
-def test_tiles_dead_half_intersection_caught():
-    # a half marked dead when not ALL its pairs are allowed (instead of none)
-    m = _mutant_dead_halves(lambda sub, lo, hi: lo > hi or not sub.all())
-    assert fails(pins.check_tiles_vs_bruteforce, m, lvsa)
-    assert fails(pins.check_tiles_half_frames, m)
-
-
-def test_tiles_dead_half_past_n_caught():
-    # forgets that a half lying wholly past N is dead
-    m = _mutant_dead_halves(lambda sub, lo, hi: lo <= hi and not sub.any())
-    assert fails(pins.check_tiles_vs_bruteforce, m, lvsa)
-    assert fails(pins.check_tiles_half_frames, m)
-
-
-def test_tiles_dead_half_swapped_caught():
-    # the two halves' bits swapped
-    m = _mutant_dead_halves(lambda sub, lo, hi: lo > hi or not sub.any())
-    orig = m.kept_tiles
-
-    def swapped(*a, **k):
-        idx, flg = orig(*a, **k)
-        return idx, [[(f & 1) | ((f & 2) << 1) | ((f & 4) >> 1) for f in r] for r in flg]
-    m.kept_tiles = swapped
-    assert fails(pins.check_tiles_vs_bruteforce, m, lvsa)
-    assert fails(pins.check_tiles_half_frames, m)
-
-
 def test_attention_transposed_operand_caught():
     m = clone(attention)
 
