@@ -357,9 +357,11 @@ def run_b200(args, rank, world, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
 
-    # the CPU-baseline pool starts (spawn) before any GPU work of this process
+    # the CPU-baseline pool starts (spawn) before any GPU work of this process;
+    # the baseline is taken at N = 1 only (rank 0 of a larger job would repeat it
+    # while every GPU of the job waits)
     pool = None
-    if rank == 0 and not args.no_cpu_baseline and not args.main_only:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.main_only:
         from oracle.pool import OraclePool
         pool = OraclePool()
 
@@ -454,8 +456,9 @@ def run_b200(args, rank, world, local):
     del qpool, o, lse, ws
     torch.cuda.empty_cache()
 
-    # ---- every other workload at full size (rank 0; replicas would only repeat it)
-    configs = run_configs(bsa, stream, peaks) if rank == 0 and not args.no_configs else None
+    # ---- every other workload at full size (N = 1 only: at N > 1 rank 0 would
+    # repeat the one-GPU figures while the other GPUs of the job are held)
+    configs = run_configs(bsa, stream, peaks) if world == 1 and not args.no_configs else None
 
     med_call = statistics.median(call_ms)
     line = {
