@@ -15,6 +15,9 @@
 // adds its rows in a fixed order before a butterfly over the lanes, so the
 // result does not depend on scheduling.  Lane j keeps the sum of the j-th
 // key tile and the warp writes its kMassKt results with one contiguous store.
+// The loads of kMassBatch key tiles are issued before any of their sums, so
+// that a warp keeps that many 512-byte loads in flight (one at a time left
+// the kernel at ~70% of HBM bandwidth: too few bytes in flight per SM).
 // Algorithmic bytes: lpart read once (H * nB * N * 4), mass written once; the
 // LSE of a row is read once per key-tile group (from L2).
 #pragma once
@@ -25,6 +28,7 @@ namespace bsa {
 constexpr int kMassThreads = 256;                  // 8 warps = 8 query blocks per CTA
 constexpr int kMassWarps = kMassThreads / 32;
 constexpr int kMassKt = 16;                        // key tiles per warp
+constexpr int kMassBatch = 4;                      // key tiles whose loads are in flight together
 
 __device__ __forceinline__ void load4(const float* p, int q0, int N, bool vec, float (&v)[4], float fill) {
   if (vec) {
@@ -59,21 +63,31 @@ blockmass_reduce_kernel(const float* __restrict__ lpart, const float* __restrict
   for (int u = 0; u < 4; ++u) l2[u] *= 1.4426950408889634f;
   const int nkt = min(kMassKt, nB - kt0);
   float keep = 0.f;
-  for (int j = 0; j < nkt; ++j) {
-    const float* lp = lpart + (static_cast<size_t>(hl) * nB + kt0 + j) * N;
-    float v[4];
-    load4(lp, q0, N, vec, v, -INFINITY);
-    float acc = 0.f;
+  for (int j0 = 0; j0 < nkt; j0 += kMassBatch) {
+    float v[kMassBatch][4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      // -inf: no allowed key of the tile in this row (or a row past N); NaN: a
-      // tile the index never reached (the workspace was set to NaN first);
-      // lse -inf: an empty row
-      if (v[u] > -INFINITY && l2[u] > -INFINITY) acc += ex2_approx(v[u] - l2[u]);
+    for (int t = 0; t < kMassBatch; ++t) {
+      if (j0 + t < nkt) {
+        load4(lpart + (static_cast<size_t>(hl) * nB + kt0 + j0 + t) * N, q0, N, vec, v[t], -INFINITY);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[t][u] = -INFINITY;
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if (lane == j) keep = acc;
+    for (int t = 0; t < kMassBatch; ++t) {
+      float acc = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        // -inf: no allowed key of the tile in this row (or a row past N); NaN:
+        // a tile the index never reached (the workspace was set to NaN first);
+        // lse -inf: an empty row
+        if (v[t][u] > -INFINITY && l2[u] > -INFINITY) acc += ex2_approx(v[t][u] - l2[u]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+      if (lane == j0 + t) keep = acc;
+    }
   }
   if (lane < nkt) mass[(static_cast<size_t>(h) * nB + qb) * nB + kt0 + lane] = keep;
 }
