@@ -551,14 +551,16 @@ def inputs_wl(wl, rank):
     return dataclasses.replace(wl, seed_base=wl.seed_base + 100000 * rank)
 
 
-def run_e2e(bsa, wl, qkv, stream, frames, counts, ix, o, lse, ws, steps, kept_tiles, world):
+def run_e2e(bsa, wl, qkv, stream, frames, counts, ix, o, lse, ws, steps, kept_tiles, world, host_out=None):
     """Same metric through the C-ABI call with pinned host buffers, as a caller
     streaming denoising steps would run it: every step copies its q, k, v
     host -> device and its o, lse device -> host inside the timed region, on
     two copy streams that overlap the attention of the neighbouring steps
     (double-buffered device inputs and outputs, ordered by events).  The
     timed region is `steps` whole steps, the first upload (before any
-    compute) and the last download (after it) included."""
+    compute) and the last download (after it) included.  With `host_out` (a
+    list), the pinned host copies of the last step's o and lse are appended
+    to it (for checking)."""
     hq, hk, hv = (x.to("cpu").pin_memory() for x in qkv)
     ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
@@ -608,6 +610,8 @@ def run_e2e(bsa, wl, qkv, stream, frames, counts, ix, o, lse, ws, steps, kept_ti
     ms = max_over_ranks(run(steps), world)
     fl = sum_over_ranks(float(sum(4 * wl.d * wl.H * kept_tiles[s % wl.T_per] * 128 * 128 for s in range(steps))),
                         world)
+    if host_out is not None:
+        host_out.extend((ho, hl))
     return {"value": fl / (ms / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms / steps, "steps": steps,
             "overlap": "copies on two streams beside the compute; first upload and last download not overlapped"}
