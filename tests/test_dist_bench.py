@@ -64,8 +64,16 @@ def test_gpus_two_starts_two_ranks():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1, r.stdout
-    assert lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
-    assert lines[0]["cpu_baseline"]["cores"] >= 1
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["cpu_baseline"]["value"] == line["value"] > 0
+    for key in ("metric", "unit", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                "dtype", "data", "config"):
+        assert key in line, key
+    assert line["config"]["workload"].startswith("tiny")
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
 
 
 @pytest.mark.timeout(300)
